@@ -1,0 +1,389 @@
+"""Benchmark of the routed-expert FP4 FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_b1|decode_b64|prefill_2048]
+
+One step = one pass of the whole path (route + w1/w3 GEMV + SwiGLU + w2 GEMV
++ combine) over one batch of fresh synthetic tokens of one DeepSeek-V4.1-Flash
+layer (hidden 5120, inter 2304, 384 experts resident in the arena, top-6).
+Inputs are resident in HBM when a timed step starts; L2 is flushed between
+timed steps (a 2x L2-sized write), so expert bytes really come from HBM.
+Rank 0 prints one JSON line.  Under torchrun each rank runs an independent
+replica (data parallel, no collective on the data path): weak scaling.
+
+``--impl reference`` times the CPU oracle (oracle/) on the host cores, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp4_routed_expert_router_b200 import synth  # noqa: E402
+
+METRIC = "MoE FP4 expert-FFN: decode HBM GB/s & tok/s (b=1); prefill TFLOP/s @2048 tok"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="decode_b1", choices=["decode_b1", "decode_b64", "prefill_2048"])
+    p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    return p.parse_args()
+
+
+def workload_config(wl: synth.Workload, graph: bool) -> dict:
+    return {
+        "workload": f"{wl.name}: one DeepSeek-V4.1-Flash routed-expert layer, {wl.notes}",
+        "hidden": wl.hidden, "inter": wl.inter, "n_experts": wl.n_experts, "top_k": wl.top_k,
+        "tokens_per_step": wl.tokens, "experts_resident": wl.n_experts,
+        "expert_bytes": wl.expert_bytes, "weights": "fp4 e2m1 + ue8m0 per 32 along K",
+        "logits": f"N(0,1) + Zipf(1.1) bias, alpha {wl.zipf_alpha}",
+        "scale_exponents": f"uniform {wl.scale_lo}..{wl.scale_hi}",
+        "l2": "flushed between timed steps (2x L2 write)",
+        "launch": "cuda graph of route+forward (PDL chain)" if graph else "eager (PDL chain)",
+        "parallelism": "replicas (one independent layer per GPU)",
+    }
+
+
+# ============================================================================ oracle arm
+def _oracle_step(wl, step, cache, n_threads):
+    """One step of the oracle: route + forward of wl.tokens fresh tokens.
+    Returns (tokens, seconds) with expert generation excluded from the time."""
+    import oracle
+    logits, _ = synth.layer_inputs(wl, 0, step)
+    x = synth.gen_x(wl.seed, wl.tokens, wl.hidden, step)
+    t0 = time.perf_counter()
+    ids, w = oracle.route(logits, wl.top_k)
+    t_route = time.perf_counter() - t0
+    objs = {}
+    for e in np.unique(ids):
+        e = int(e)
+        if e not in cache:
+            cache[e] = synth.expert_object(synth.gen_expert(wl.seed, 0, e, wl.hidden, wl.inter, wl.scale_lo,
+                                                            wl.scale_hi), wl.hidden, wl.inter)
+        objs[e] = cache[e]
+    t1 = time.perf_counter()
+    oracle.moe_forward(x, ids, w, objs, wl.n_experts, wl.hidden, wl.inter, n_threads=n_threads)
+    return wl.tokens, t_route + time.perf_counter() - t1
+
+
+def cpu_baseline(wl: synth.Workload, budget_s: float = 15.0, max_steps: int = 64) -> dict:
+    """The oracle timed on this host's cores on a bounded sample of the workload."""
+    import oracle
+    n_threads = oracle.max_threads()
+    if wl.tokens > 8:   # sample 8-token batches of the big workloads
+        wl = synth.Workload(**{**wl.__dict__, "tokens": 8})
+    cache, toks, secs, steps = {}, 0, 0.0, 0
+    while steps < max_steps and secs < budget_s:
+        n, s = _oracle_step(wl, 10_000 + steps, cache, n_threads)
+        toks += n
+        secs += s
+        steps += 1
+    return {"value": toks / secs, "unit": "tok/s", "cores": n_threads, "kind": "oracle",
+            "sample": f"{steps} steps x {wl.tokens} token(s) of {wl.name} (fp64 oracle, OpenMP over "
+                      f"(token, expert) pairs, expert generation excluded), {secs:.1f} s"}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    n_threads = oracle.max_threads()
+    swl = wl if wl.tokens <= 8 else synth.Workload(**{**wl.__dict__, "tokens": 8})
+    cache = {}
+    for i in range(args.warmup):
+        _oracle_step(swl, 20_000 + i, cache, n_threads)
+    toks, secs = 0, 0.0
+    for i in range(args.steps):
+        n, s = _oracle_step(swl, 30_000 + i, cache, n_threads)
+        toks += n
+        secs += s
+    value = toks / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, False),
+            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": n_threads, "kind": "oracle",
+                             "sample": f"{args.steps} steps x {swl.tokens} token(s) of {wl.name}"},
+            "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ============================================================================ GPU arm
+class ClockSampler:
+    """SM clock and throttle-reason sampling DURING the timed region: an NVML
+    reader thread polling every ~0.5 ms (read-only queries), with nvidia-smi
+    as a fallback when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = False
+
+    def _poll(self, nv, h):
+        masks = [(n, getattr(nv, c, 0)) for n, c in self.REASONS]
+        while not self._stop:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for n, m in masks:
+                    if m and (r & m):
+                        self.reasons.add(n)
+            except Exception:
+                break
+            time.sleep(0.0005)
+
+    def __enter__(self):
+        import threading
+        self._thread = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+        return self
+
+    def _physical_index(self) -> int:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[self.idx])
+            except (ValueError, IndexError):
+                pass
+        return self.idx
+
+    def __exit__(self, *exc):
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def measured_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+    from fp4_routed_expert_router_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # ---- arena: every expert of the layer resident, generated on the device
+    T = wl.tokens
+    ctx = moe.Context(wl.hidden, wl.inter, wl.n_experts, wl.top_k, 1, wl.n_experts, max(T, 8), device=local)
+    staging = torch.empty(wl.expert_bytes, dtype=torch.uint8, device=dev)
+    for e in range(wl.n_experts):
+        moe.synth_fill_expert(staging, wl.seed, 0, e, wl.hidden, wl.inter, wl.scale_lo, wl.scale_hi)
+        ctx.load_expert_object(0, e, e, staging)
+    torch.cuda.synchronize()
+    rc, msg = ctx.last_error()
+    assert rc == moe.OK, msg
+
+    # ---- a pool of fresh inputs resident in HBM (different per rank)
+    npool = 64
+    pool_x = torch.empty((npool, T, wl.hidden), dtype=torch.int16, device=dev)
+    pool_l = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, device=dev)
+    for i in range(npool):
+        st = rank * 100_000 + i
+        pool_x[i] = torch.from_numpy(synth.gen_x(wl.seed, T, wl.hidden, st).view(np.int16))
+        pool_l[i] = torch.from_numpy(synth.layer_inputs(wl, 0, st)[0])
+    x_buf = torch.empty((T, wl.hidden), dtype=torch.int16, device=dev)
+    l_buf = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
+    y_buf = torch.empty((T, wl.hidden), dtype=torch.float32, device=dev)
+    routing = ctx.alloc_routing(T)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_launch():
+        ctx.route(0, l_buf, out=routing, stream=stream)
+        ctx.forward(0, x_buf, routing, y=y_buf, stream=stream)
+
+    def stage(i):
+        x_buf.copy_(pool_x[i % npool], non_blocking=True)
+        l_buf.copy_(pool_l[i % npool], non_blocking=True)
+        flush.fill_(float(i))
+
+    graph = None
+    with torch.cuda.stream(stream):
+        stage(0)
+        step_launch()
+        stream.synchronize()
+        if not args.no_graph:
+            try:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    step_launch()
+                graph = g
+            except Exception as ex:  # graph capture unavailable: launch eagerly
+                print(f"# cuda graph capture failed ({ex}); launching eagerly", file=sys.stderr)
+                graph = None
+        run = graph.replay if graph is not None else step_launch
+
+        for i in range(args.warmup):
+            stage(i)
+            run()
+        stream.synchronize()
+        rc, msg = ctx.last_error()
+        assert rc == moe.OK, msg
+
+        # ---- timed region: K steps, events on the launching stream, L2 flushed between steps
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            for i in range(args.steps):
+                stage(1000 + i)
+                ev[i][0].record(stream)
+                run()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        total_ms = sum(step_ms)
+
+        # ---- per-kernel pass: same steps, events around every kernel
+        ctx.set_profile(True)
+        ctx.profile_read()
+        n_active = []
+        for i in range(args.steps):
+            stage(1000 + i)
+            step_launch()
+            n_active.append(int((routing.counts > 0).sum()))
+        recs = ctx.profile_read()
+        ctx.set_profile(False)
+
+        # ---- end to end through the public API with host buffers
+        hx = torch.empty((npool, T, wl.hidden), dtype=torch.int16, pin_memory=True)
+        hl = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, pin_memory=True)
+        hx.copy_(pool_x.cpu())
+        hl.copy_(pool_l.cpu())
+        hy = torch.empty((T, wl.hidden), dtype=torch.float32, pin_memory=True)
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            e2e_ev[i][0].record(stream)
+            x_buf.copy_(hx[i % npool], non_blocking=True)
+            l_buf.copy_(hl[i % npool], non_blocking=True)
+            run()
+            hy.copy_(y_buf, non_blocking=True)
+            e2e_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    rc, msg = ctx.last_error()
+    assert rc == moe.OK, msg
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    # ---- roofline of the dominant kernel (w1/w3 stream)
+    per_kernel = {}
+    for name, ms in recs:
+        per_kernel.setdefault(name, []).append(ms)
+    avg = {k: sum(v) / len(v) for k, v in per_kernel.items()}
+    peaks, peak_src = measured_peaks()
+    E, H, I, k = wl.n_experts, wl.hidden, wl.inter, wl.top_k
+    up_bytes_expert = 2 * (I * H // 2 + I * H // 32)
+    down_bytes_expert = H * I // 2 + H * I // 32
+    act = float(np.mean(n_active))   # active experts per step, from the routing counts
+    dominant = "gemv_up" if "gemv_up" in avg else max(avg, key=avg.get)
+    dom_bytes = act * (up_bytes_expert if dominant == "gemv_up" else down_bytes_expert)
+    achieved = dom_bytes / (avg[dominant] * 1e-3) / 1e9
+    layer_bytes = act * (up_bytes_expert + down_bytes_expert)
+    fwd_ms = sum(avg.get(n, 0.0) for n in ("gemv_up", "gemv_down", "combine"))
+
+    ms_per_step = total_ms / args.steps
+    toks = T * args.steps * world
+    value = toks / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, graph is not None),
+        "hbm_gbs_step": layer_bytes / (ms_per_step * 1e-3) / 1e9,
+        "hbm_frac_step": layer_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "kernel_ms": avg,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs",
+                     "algorithmic_bytes_per_launch": dom_bytes},
+        "layer_roofline": {"bytes_per_step": layer_bytes, "forward_kernels_ms": fwd_ms,
+                           "achieved_gbs": layer_bytes / (fwd_ms * 1e-3) / 1e9 if fwd_ms else None,
+                           "frac": (layer_bytes / (fwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if fwd_ms else None},
+        "active_experts_per_step": act,
+        "e2e": {"value": toks / (e2e_ms * 1e-3), "unit": "tok/s",
+                "h2d_bytes_per_step": T * (wl.hidden * 2 + wl.n_experts * 4),
+                "d2h_bytes_per_step": T * wl.hidden * 4},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,444 @@
+// moe_fp4_api.cu -- C ABI of libmoe_fp4 (declared in include/moe_fp4.h):
+// context, HBM expert arena with its (layer, expert) -> slot table, slot
+// loading, routing and the expert FFN forward.  All compute runs in the CUDA
+// kernels of csrc/*.cuh; there is no host-side arithmetic on the data path and
+// no CPU fallback.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/moe_fp4.h"
+#include "common.cuh"
+#include "decode_gemv.cuh"
+#include "fp4_decode.cuh"
+#include "router.cuh"
+#include "tc_prefill.cuh"
+
+using namespace moe;
+
+struct moe_fp4_ctx {
+    moe_fp4_config cfg{};
+    int device = 0;
+    int sm_count = 0;
+    size_t slot_bytes = 0;
+    size_t off_w3 = 0, off_w2 = 0, off_s1 = 0, off_s3 = 0, off_s2 = 0;
+    uint8_t* arena = nullptr;
+    bool own_arena = false;
+    int32_t* d_table = nullptr;        // [L][E]
+    uint8_t* d_staging = nullptr;      // one expert, checkpoint layout
+    uint16_t* d_h = nullptr;           // [max_tokens*k, I] bf16
+    float* d_o = nullptr;              // [max_tokens*k, H] fp32
+    int* d_err = nullptr;              // error word [4]
+    unsigned int* d_ticket = nullptr;  // route kernel ticket
+    std::vector<int32_t> h_table;      // host mirror of d_table
+    std::vector<int64_t> slot_owner;   // slot -> layer*E+expert or -1
+    int path = MOE_FP4_PATH_AUTO;
+    bool profile = false;
+    struct ProfRec { const char* name; cudaEvent_t a, b; };
+    std::vector<ProfRec> prof;         // profiled launches not yet read
+    std::vector<cudaEvent_t> ev_free;  // recycled events
+    TcPlan tc{};                       // tcgen05 prefill workspace
+    std::string host_msg;
+    moe_fp4_status host_status = MOE_FP4_OK;
+};
+
+namespace {
+
+moe_fp4_status host_fail(moe_fp4_ctx* c, moe_fp4_status s, const char* fmt, ...) {
+    if (c) {
+        char buf[256];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        c->host_msg = buf;
+        c->host_status = s;
+    }
+    return s;
+}
+
+moe_fp4_status cuda_fail(moe_fp4_ctx* c, cudaError_t e, const char* what) {
+    return host_fail(c, MOE_FP4_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool config_ok(const moe_fp4_config* c) {
+    if (!c) return false;
+    if (c->hidden <= 0 || c->inter <= 0 || c->hidden % 128 || c->inter % 128) return false;
+    if (c->n_experts <= 0 || c->n_experts > 1024) return false;
+    if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->n_experts) return false;
+    if (c->n_layers <= 0 || c->n_slots <= 0 || c->max_tokens <= 0) return false;
+    if (static_cast<long long>(c->max_tokens) * c->top_k > (1LL << 30)) return false;
+    return true;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+cudaEvent_t take_event(moe_fp4_ctx* c) {
+    if (!c->ev_free.empty()) {
+        cudaEvent_t e = c->ev_free.back();
+        c->ev_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Launch with programmatic dependent launch; bracket with events when the
+// context profiles (at most 65536 pending records are kept).
+template <typename Kern, typename... Args>
+cudaError_t launch_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, Args... args) {
+    const bool prof = c->profile && c->prof.size() < 65536;
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    if (prof) {
+        ea = take_event(c);
+        eb = take_event(c);
+        cudaEventRecord(ea, s);
+    }
+    cudaError_t e = launch_pdl(kern, grid, block, smem, s, args...);
+    if (prof) {
+        cudaEventRecord(eb, s);
+        c->prof.push_back({name, ea, eb});
+    }
+    return e;
+}
+
+// Re-encode the code words of one expert (staging, checkpoint layout) into
+// its slot, copy the scales, check every scale byte is in [2, 252], and map
+// the slot.  One thread per 32-bit word of codes / per 4 scale bytes.
+__global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                 size_t code_words, size_t scale_bytes, int32_t* table,
+                                 int map_index, int slot, int* err) {
+    const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src);
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
+    if (i < code_words) {
+        d32[i] = fp4_reencode_word(s32[i]);
+    } else if (i < code_words + (scale_bytes + 3) / 4) {
+        const size_t b0 = (i - code_words) * 4;
+        for (size_t b = b0; b < b0 + 4 && b < scale_bytes; ++b) {
+            const uint8_t v = src[code_words * 4 + b];
+            dst[code_words * 4 + b] = v;
+            if (v < 2 || v > 252) latch_error(err, ERR_EINVAL, static_cast<int>(b), KID_LOAD);
+        }
+    }
+    if (i == 0 && map_index >= 0) table[map_index] = slot;
+}
+
+const char* kernel_name(int kid) {
+    switch (kid) {
+        case KID_ROUTE: return "route";
+        case KID_LOAD: return "load_expert_slot";
+        case KID_UP: return "gemv_up";
+        case KID_DOWN: return "gemv_down";
+        case KID_COMBINE: return "combine";
+        case KID_TC_UP: return "tc_up";
+        case KID_TC_DOWN: return "tc_down";
+        case KID_GATHER: return "gather";
+        default: return "?";
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_fp4_slot_bytes(const moe_fp4_config* cfg) {
+    if (!config_ok(cfg)) return 0;
+    const size_t H = cfg->hidden, I = cfg->inter;
+    return 2 * (I * H / 2 + I * H / 32) + (H * I / 2 + H * I / 32);
+}
+
+moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena,
+                              size_t arena_bytes, moe_fp4_ctx** out) {
+    if (!out) return MOE_FP4_EINVAL;
+    *out = nullptr;
+    if (!config_ok(cfg)) return MOE_FP4_EINVAL;
+    moe_fp4_ctx* c = new moe_fp4_ctx();
+    c->cfg = *cfg;
+    c->device = device;
+    const size_t H = cfg->hidden, I = cfg->inter, E = cfg->n_experts, L = cfg->n_layers;
+    c->slot_bytes = moe_fp4_slot_bytes(cfg);
+    c->off_w3 = I * H / 2;
+    c->off_w2 = I * H;
+    c->off_s1 = I * H + H * I / 2;
+    c->off_s3 = c->off_s1 + I * H / 32;
+    c->off_s2 = c->off_s3 + I * H / 32;
+    const size_t need = c->slot_bytes * static_cast<size_t>(cfg->n_slots);
+    auto bail = [&](moe_fp4_status s) {
+        moe_fp4_destroy(c);
+        return s;
+    };
+    if (arena && (arena_bytes < need || (reinterpret_cast<uintptr_t>(arena) & 255))) return bail(MOE_FP4_EINVAL);
+    cudaError_t e = cudaSetDevice(device);
+    if (e != cudaSuccess) return bail(MOE_FP4_ECUDA);
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+    cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
+    if (major < 10) return bail(MOE_FP4_ECUDA);   // sm_100a code only
+    if (arena) {
+        c->arena = static_cast<uint8_t*>(arena);
+    } else {
+        if (cudaMalloc(&c->arena, need) != cudaSuccess) { cudaGetLastError(); return bail(MOE_FP4_ENOMEM); }
+        c->own_arena = true;
+    }
+    const size_t ent = static_cast<size_t>(cfg->max_tokens) * cfg->top_k;
+    if (cudaMalloc(&c->d_table, sizeof(int32_t) * L * E) != cudaSuccess ||
+        cudaMalloc(&c->d_staging, c->slot_bytes) != cudaSuccess ||
+        cudaMalloc(&c->d_h, sizeof(uint16_t) * ent * I) != cudaSuccess ||
+        cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
+        cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
+        cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
+        cudaGetLastError();
+        return bail(MOE_FP4_ENOMEM);
+    }
+    if (tc_plan_create(&c->tc, *cfg) != cudaSuccess) { cudaGetLastError(); return bail(MOE_FP4_ENOMEM); }
+    if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
+        cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
+        cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
+        return bail(MOE_FP4_ECUDA);
+    c->h_table.assign(L * E, -1);
+    c->slot_owner.assign(cfg->n_slots, -1);
+    *out = c;
+    return MOE_FP4_OK;
+}
+
+void moe_fp4_destroy(moe_fp4_ctx* c) {
+    if (!c) return;
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    if (c->own_arena) cudaFree(c->arena);
+    cudaFree(c->d_table);
+    cudaFree(c->d_staging);
+    cudaFree(c->d_h);
+    cudaFree(c->d_o);
+    cudaFree(c->d_err);
+    cudaFree(c->d_ticket);
+    tc_plan_destroy(&c->tc);
+    for (auto& r : c->prof) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+    for (auto e : c->ev_free) cudaEventDestroy(e);
+    delete c;
+}
+
+void* moe_fp4_arena(moe_fp4_ctx* c) { return c ? c->arena : nullptr; }
+
+moe_fp4_status moe_fp4_set_option(moe_fp4_ctx* c, int option, int value) {
+    if (!c) return MOE_FP4_EINVAL;
+    if (option == MOE_FP4_OPT_PATH && value >= MOE_FP4_PATH_AUTO && value <= MOE_FP4_PATH_TC) {
+        c->path = value;
+        return MOE_FP4_OK;
+    }
+    if (option == MOE_FP4_OPT_PROFILE && (value == 0 || value == 1)) {
+        c->profile = value != 0;
+        return MOE_FP4_OK;
+    }
+    return host_fail(c, MOE_FP4_EINVAL, "set_option: unknown option %d / value %d", option, value);
+}
+
+moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx* c, int layer, int expert, int slot,
+                                        const uint8_t* w1, const uint8_t* w1_scale,
+                                        const uint8_t* w3, const uint8_t* w3_scale,
+                                        const uint8_t* w2, const uint8_t* w2_scale, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || expert < 0 || expert >= g.n_experts || slot < -1 || slot >= g.n_slots)
+        return host_fail(c, MOE_FP4_EINVAL, "load_expert_slot: layer %d expert %d slot %d out of range",
+                         layer, expert, slot);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int idx = layer * g.n_experts + expert;
+    cudaError_t e;
+    // release what (layer, expert) and `slot` were bound to
+    const int old_slot = c->h_table[idx];
+    if (old_slot >= 0) c->slot_owner[old_slot] = -1;
+    c->h_table[idx] = -1;
+    if (slot == -1) {
+        e = cudaMemsetAsync(c->d_table + idx, 0xFF, sizeof(int32_t), s);
+        return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "load_expert_slot: unmap");
+    }
+    if (!w1 || !w1_scale || !w3 || !w3_scale || !w2 || !w2_scale)
+        return host_fail(c, MOE_FP4_EINVAL, "load_expert_slot: NULL tensor");
+    const int64_t prev = c->slot_owner[slot];
+    if (prev >= 0) {
+        c->h_table[prev] = -1;
+        e = cudaMemsetAsync(c->d_table + prev, 0xFF, sizeof(int32_t), s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: evict");
+    }
+    const size_t H = g.hidden, I = g.inter;
+    const struct { const uint8_t* p; size_t off, n; } parts[6] = {
+        {w1, 0, I * H / 2},          {w3, c->off_w3, I * H / 2},       {w2, c->off_w2, H * I / 2},
+        {w1_scale, c->off_s1, I * H / 32}, {w3_scale, c->off_s3, I * H / 32}, {w2_scale, c->off_s2, H * I / 32}};
+    for (const auto& p : parts) {
+        e = cudaMemcpyAsync(c->d_staging + p.off, p.p, p.n, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: copy");
+    }
+    const size_t code_words = c->off_s1 / 4, scale_bytes = c->slot_bytes - c->off_s1;
+    const size_t threads = code_words + (scale_bytes + 3) / 4;
+    load_slot_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
+        c->d_staging, c->arena + static_cast<size_t>(slot) * c->slot_bytes, code_words, scale_bytes,
+        c->d_table, idx, slot, c->d_err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: launch");
+    c->h_table[idx] = slot;
+    c->slot_owner[slot] = idx;
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_route(moe_fp4_ctx* c, int layer, const float* logits, const uint8_t* keep_mask,
+                             int T, int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || T < 0 || T > g.max_tokens)
+        return host_fail(c, MOE_FP4_EINVAL, "route: layer %d / T %d out of range", layer, T);
+    if ((T > 0 && (!logits || !ids || !weights || !perm)) || !counts || !offsets)
+        return host_fail(c, MOE_FP4_EINVAL, "route: NULL output");
+    RouteArgs a{logits, keep_mask, T, g.n_experts, g.top_k, ids, weights, counts, offsets, perm,
+                c->d_ticket, c->d_err};
+    const unsigned grid = T > 0 ? static_cast<unsigned>((T + kRouteWarps - 1) / kRouteWarps) : 1u;
+    const size_t smem = sizeof(int) * kRouteWarps * g.n_experts;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (g.n_experts <= 128)
+        e = launch_k(c, "route", route_kernel<4>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+    else if (g.n_experts <= 384)
+        e = launch_k(c, "route", route_kernel<12>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+    else
+        e = launch_k(c, "route", route_kernel<32>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+    return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "route: launch");
+}
+
+static int pick_warps(int nchunks) {
+    for (int w : {8, 6, 4, 2, 1})
+        if (nchunks % w == 0) return w;
+    return 8;
+}
+
+static cudaError_t launch_up(moe_fp4_ctx* c, int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
+    switch (nw) {
+        case 1: return launch_k(c, "gemv_up", gemv_up_kernel<1>, grid, dim3(32), 0, s, a);
+        case 2: return launch_k(c, "gemv_up", gemv_up_kernel<2>, grid, dim3(64), 0, s, a);
+        case 4: return launch_k(c, "gemv_up", gemv_up_kernel<4>, grid, dim3(128), 0, s, a);
+        case 6: return launch_k(c, "gemv_up", gemv_up_kernel<6>, grid, dim3(192), 0, s, a);
+        default: return launch_k(c, "gemv_up", gemv_up_kernel<8>, grid, dim3(256), 0, s, a);
+    }
+}
+static cudaError_t launch_down(moe_fp4_ctx* c, int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
+    switch (nw) {
+        case 1: return launch_k(c, "gemv_down", gemv_down_kernel<1>, grid, dim3(32), 0, s, a);
+        case 2: return launch_k(c, "gemv_down", gemv_down_kernel<2>, grid, dim3(64), 0, s, a);
+        case 4: return launch_k(c, "gemv_down", gemv_down_kernel<4>, grid, dim3(128), 0, s, a);
+        case 6: return launch_k(c, "gemv_down", gemv_down_kernel<6>, grid, dim3(192), 0, s, a);
+        default: return launch_k(c, "gemv_down", gemv_down_kernel<8>, grid, dim3(256), 0, s, a);
+    }
+}
+
+moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int T, const int32_t* ids,
+                               const float* weights, const int32_t* counts, const int32_t* offsets,
+                               const int32_t* perm, float* y, uint16_t* x_out, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || T < 0 || T > g.max_tokens)
+        return host_fail(c, MOE_FP4_EINVAL, "forward: layer %d / T %d out of range", layer, T);
+    if (T == 0) return MOE_FP4_OK;
+    if (!x || !ids || !weights || !counts || !offsets || !perm || !y)
+        return host_fail(c, MOE_FP4_EINVAL, "forward: NULL argument");
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
+        (reinterpret_cast<uintptr_t>(x_out) & 7) || (reinterpret_cast<uintptr_t>(weights) & 3))
+        return host_fail(c, MOE_FP4_EINVAL, "forward: x and y must be 16-byte aligned, x_out 8-byte");
+    (void)ids;
+    (void)counts;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int H = g.hidden, I = g.inter, E = g.n_experts, k = g.top_k;
+    const int ent = T * k;
+    const int active_max = ent < E ? ent : E;
+    GemvArgs a{c->arena, c->slot_bytes, c->off_w3, c->off_w2, c->off_s1, c->off_s3, c->off_s2,
+               c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_h, c->d_o, c->d_err};
+    bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
+    cudaError_t e;
+    if (use_tc) {
+        e = tc_forward(&c->tc, a, T, s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "forward: tc launch");
+    } else {
+        e = launch_up(c, pick_warps(H / 128), dim3(I / 16, active_max), s, a);
+        if (e != cudaSuccess) return cuda_fail(c, e, "forward: up launch");
+        e = launch_down(c, pick_warps(I / 128), dim3(H / 16, active_max), s, a);
+        if (e != cudaSuccess) return cuda_fail(c, e, "forward: down launch");
+    }
+    const int n4 = T * (H / 4);
+    e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
+                 static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
+    if (e != cudaSuccess) return cuda_fail(c, e, "forward: combine launch");
+    return MOE_FP4_OK;
+}
+
+int moe_fp4_profile_read(moe_fp4_ctx* c, const char** names, float* ms, int max) {
+    if (!c) return -1;
+    cudaSetDevice(c->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    int n = 0;
+    for (const auto& r : c->prof) {
+        if (n < max) {
+            float t = 0.f;
+            if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return -1;
+            if (names) names[n] = r.name;
+            if (ms) ms[n] = t;
+            ++n;
+        }
+        c->ev_free.push_back(r.a);
+        c->ev_free.push_back(r.b);
+    }
+    c->prof.clear();
+    return n;
+}
+
+moe_fp4_status moe_fp4_last_error(moe_fp4_ctx* c, char* msg, size_t n) {
+    if (!c) return MOE_FP4_EINVAL;
+    cudaSetDevice(c->device);
+    std::string text;
+    moe_fp4_status st = MOE_FP4_OK;
+    cudaError_t e = cudaDeviceSynchronize();
+    int w[4] = {0, 0, 0, 0};
+    if (e == cudaSuccess) e = cudaMemcpy(w, c->d_err, sizeof w, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof w);
+    if (e != cudaSuccess) {
+        st = MOE_FP4_ECUDA;
+        text = std::string("cuda: ") + cudaGetErrorString(e);
+    } else if (w[0] != 0) {
+        st = static_cast<moe_fp4_status>(w[0]);
+        char buf[160];
+        const char* what = w[0] == ERR_ESLOT ? "expert has no slot" : w[0] == ERR_ETIMEOUT ? "wait timed out"
+                                                                                           : "invalid data";
+        snprintf(buf, sizeof buf, "%s (kernel %s, detail %d)", what, kernel_name(w[2]), w[1]);
+        text = buf;
+    } else if (c->host_status != MOE_FP4_OK) {
+        st = c->host_status;
+        text = c->host_msg;
+    }
+    c->host_status = MOE_FP4_OK;
+    c->host_msg.clear();
+    if (msg && n) {
+        snprintf(msg, n, "%s", text.c_str());
+    }
+    return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+// router.cuh -- top-k routing and token->expert grouping in one launch.
+//
+// Router: 6 of 384 routed experts per token per layer (10100.com article
+// 151357339, section "moe专家的容量瓶颈"); the function itself is not given
+// on the pages.  It is read as softmax over fp32 logits, top-k under the
+// total order (larger logit first, lower expert index on ties, -0 == +0),
+// renormalised over the k chosen: w_j = exp(l_j - l_max) / sum_i exp(l_i - l_max).
+// Experts outside the layer's keep mask are never chosen (section "方案二").
+//
+// Grouping: in prefill one read of an expert's weights serves every token
+// routed to it (ai-shiz.ru "DeepSeek-V4.1-Flash дома", trick 4).  The
+// entries t*k+j are grouped by expert with a stable counting sort: per-warp
+// histograms with warp-aggregated updates (match_any), an exclusive scan,
+// and a second, ordered pass that places each entry.
+//
+// Launch: one warp per token, 8 tokens per CTA.  The CTA that finishes last
+// (a release/acquire ticket) runs the grouping over all T*k entries, so route
+// is a single kernel whatever T is.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouteWarps = 8;
+
+// Order-preserving map of a float (after -0 -> +0) to uint32; 0 is below
+// every real value and marks "not selectable".
+__device__ __forceinline__ uint32_t orderable(float v) {
+    uint32_t b = __float_as_uint(v + 0.0f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_orderable(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+struct RouteArgs {
+    const float* logits;
+    const uint8_t* keep;
+    int T, E, k;
+    int32_t* ids;
+    float* weights;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm;
+    unsigned int* ticket;   // zero between launches
+    int* err;
+};
+
+template <int NI>   // logits held per lane: E <= 32 * NI
+__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane) {
+    const float* l = a.logits + static_cast<size_t>(t) * a.E;
+    uint32_t key[NI];
+    bool nan = false;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        int e = lane + 32 * i;
+        key[i] = 0;
+        if (e < a.E) {
+            float v = __ldg(l + e);
+            nan |= (v != v);
+            bool ok = (a.keep == nullptr) || (__ldg(a.keep + e) != 0);
+            key[i] = ok ? orderable(v) : 0u;
+        }
+    }
+    if (__any_sync(0xFFFFFFFFu, nan)) {
+        if (lane == 0) latch_error(a.err, ERR_EINVAL, t, KID_ROUTE);
+    }
+    uint32_t removed = 0;
+    int my_id = 0;
+    float my_val = 0.f;
+    bool short_of_experts = false;
+    for (int r = 0; r < a.k; ++r) {
+        uint32_t best = 0;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            uint32_t kk = (removed >> i) & 1u ? 0u : key[i];
+            if (kk > best) { best = kk; bi = i; }
+        }
+        uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, best);
+        uint32_t cand = (best == wmax) ? static_cast<uint32_t>(lane + 32 * bi) : 0xFFFFFFFFu;
+        uint32_t win = __reduce_min_sync(0xFFFFFFFFu, cand);
+        if (wmax == 0u) { short_of_experts = true; win = 0; }
+        if ((win & 31u) == static_cast<uint32_t>(lane)) removed |= 1u << (win >> 5);
+        if (lane == r) { my_id = static_cast<int>(win); my_val = from_orderable(wmax); }
+    }
+    if (short_of_experts) {
+        if (lane == 0) latch_error(a.err, ERR_EINVAL, t, KID_ROUTE);
+    }
+    float lmax = __shfl_sync(0xFFFFFFFFu, my_val, 0);
+    float p = (lane < a.k) ? expf(my_val - lmax) : 0.0f;
+    float s = p;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    if (lane < a.k) {
+        a.ids[static_cast<size_t>(t) * a.k + lane] = my_id;
+        a.weights[static_cast<size_t>(t) * a.k + lane] = p / s;
+    }
+}
+
+// Stable grouping of all T*k entries by one CTA of kRouteWarps warps.
+// smem: int hist[kRouteWarps][E].
+__device__ void group_entries(const RouteArgs& a, int* hist) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NE = a.T * a.k, E = a.E;
+    for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int seg = (NE + kRouteWarps - 1) / kRouteWarps;
+    const int lo = min(NE, warp * seg), hi = min(NE, lo + seg);
+    int* h = hist + warp * E;
+    // pass 1: per-warp histogram, one update per distinct expert of a batch
+    for (int b = lo; b < hi; b += 32) {
+        int i = b + lane;
+        int e = (i < hi) ? ld_cg(a.ids + i) : -1;
+        if (e >= E || (i < hi && e < 0)) { latch_error(a.err, ERR_EINVAL, i, KID_ROUTE); e = -1; }
+        uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+    }
+    __syncthreads();
+    // exclusive scan of counts over experts (warp 0), then per-warp bases
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        int local = 0;
+        for (int q = 0; q < per; ++q) {
+            int e = lane * per + q;
+            if (e < E) for (int w = 0; w < kRouteWarps; ++w) local += hist[w * E + e];
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int q = 0; q < per; ++q) {
+            int e = lane * per + q;
+            if (e < E) {
+                int c = 0;
+                a.offsets[e] = run;
+                for (int w = 0; w < kRouteWarps; ++w) {
+                    int v = hist[w * E + e];
+                    hist[w * E + e] = run + c;
+                    c += v;
+                }
+                a.counts[e] = c;
+                run += c;
+            }
+        }
+        if (lane == 31) a.offsets[E] = run;
+    }
+    __syncthreads();
+    // pass 2: place entries in order
+    for (int b = lo; b < hi; b += 32) {
+        int i = b + lane;
+        int e = (i < hi) ? ld_cg(a.ids + i) : -1;
+        if (e >= E) e = -1;
+        uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+        int base = (e >= 0) ? h[e] : 0;
+        __syncwarp();
+        if (e >= 0) {
+            a.perm[base + __popc(peers & lanemask_lt())] = i;
+            if (lane == __ffs(peers) - 1) h[e] = base + __popc(peers);
+        }
+        __syncwarp();
+    }
+}
+
+template <int NI>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
+    extern __shared__ int smem_hist[];
+    __shared__ int is_last;
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kRouteWarps + warp;
+    if (t < a.T) route_token<NI>(a, t, lane);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned int prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.ticket) : "memory");
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    group_entries(a, smem_hist);
+    pdl_trigger();
+    if (threadIdx.x == 0) *a.ticket = 0;
+}
+
+}  // namespace moe

@@ -1,0 +1,198 @@
+/*
+ * moe_fp4.h -- C ABI of the routed-expert FP4 FFN library (libmoe_fp4.so).
+ *
+ * One MoE layer of the DeepSeek-V4.1-Flash shape: hidden 5120, expert
+ * intermediate 2304, 384 routed experts, top-6 per token (10100.com article
+ * 151357339, section "moe专家的容量瓶颈").  Experts live in an HBM arena of
+ * fixed-size slots addressed through a (layer, expert) -> slot table, the
+ * "Expert Arena" of the same article (section "方案一：hot expert常驻内存").
+ *
+ * The layer computes, per token t:
+ *   router   ids[t, 0..k) = top-k of the fp32 logits (larger first, lower
+ *            expert index on ties), w[t, j] = softmax renormalised over them;
+ *   permute  the (t, j) entries grouped by expert;
+ *   expert   a1 = x W1^T, a3 = x W3^T, h = bf16(silu(a1) * a3), o = h W2^T
+ *            with W = E2M1 code * 2^(UE8M0 - 127), one scale per 32 along K;
+ *   combine  y[t] = sum_j w[t, j] * o[t, j].
+ * The router function, the activation and the nibble order are not fixed by
+ * the pages; this library reads them as above (softmax + renormalise,
+ * SwiGLU with w1 = gate and w3 = up, low nibble = even K index).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller unless a
+ *    parameter says "host or device".  Layouts are row-major and dense.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls that launch work are asynchronous on that stream; their
+ *    status reports argument checks and launch errors only.  Errors found by
+ *    kernels (an expert with no slot, a NaN logit, a scale outside the
+ *    supported range) are latched in a device error word and reported by
+ *    moe_fp4_last_error.  No kernel traps; there is no CPU fallback.
+ *  - A context is bound to one device; calls must be made with that device
+ *    current.  A context is not thread-safe.
+ */
+#ifndef MOE_FP4_H
+#define MOE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_fp4_ctx moe_fp4_ctx;
+
+typedef enum {
+    MOE_FP4_OK = 0,
+    MOE_FP4_EINVAL = 1,   /* bad argument, shape, NaN logit or bad scale byte */
+    MOE_FP4_ENOMEM = 2,   /* device allocation failed */
+    MOE_FP4_ECUDA = 3,    /* a CUDA runtime call or launch failed */
+    MOE_FP4_ESLOT = 4,    /* a routed (layer, expert) has no arena slot */
+    MOE_FP4_ETIMEOUT = 5  /* a bounded device-side wait gave up */
+} moe_fp4_status;
+
+typedef struct {
+    int32_t hidden;      /* H: model width (5120); multiple of 128 */
+    int32_t inter;       /* I: expert intermediate width (2304); multiple of 128 */
+    int32_t n_experts;   /* E: routed experts per layer (384); <= 1024 */
+    int32_t top_k;       /* k: experts per token (6); 1 <= k <= min(E, 32) */
+    int32_t n_layers;    /* L: layers addressed by the slot table */
+    int32_t n_slots;     /* arena capacity in expert slots */
+    int32_t max_tokens;  /* largest T accepted by route / forward */
+} moe_fp4_config;
+
+/* Execution-path override for moe_fp4_set_option(MOE_FP4_OPT_PATH, .). */
+enum {
+    MOE_FP4_PATH_AUTO = 0,  /* grouped GEMV for small batches, tcgen05 GEMM above */
+    MOE_FP4_PATH_GEMV = 1,  /* always the register-decoded grouped GEMV */
+    MOE_FP4_PATH_TC = 2     /* always the tcgen05 grouped GEMM */
+};
+/* Options for moe_fp4_set_option. */
+enum {
+    MOE_FP4_OPT_PATH = 1,     /* value: MOE_FP4_PATH_* */
+    MOE_FP4_OPT_PROFILE = 2   /* value 1: time every kernel with CUDA events */
+};
+
+/*
+ * Bytes of one expert slot: 2*(I*H/2 + I*H/32) + (H*I/2 + H*I/32); for the
+ * V4.1 shape 18,800,640 (10100.com article, section "moe专家的容量瓶颈").
+ * Returns 0 for an invalid config.
+ *
+ * Slot layout (offsets from the slot base, all multiples of 128 bytes for
+ * the V4.1 shape): w1 codes [I, H/2] at 0, w3 codes at I*H/2, w2 codes
+ * [H, I/2] at I*H, then s1 [I, H/32], s3 [I, H/32], s2 [H, I/32] scales:
+ * codes first, scales after, as the article stores the expert object
+ * (section "SSD读取性能").  Inside the slot each 32-bit word of codes is
+ * re-encoded by moe_fp4_load_expert_slot (the eight sign bits are moved so
+ * that the in-register decoder of csrc/fp4_decode.cuh needs fewer
+ * instructions; magnitudes stay in place); scales are stored as is.
+ */
+size_t moe_fp4_slot_bytes(const moe_fp4_config *cfg);
+
+/*
+ * Create a context on `device`.
+ *  arena:       device pointer to at least n_slots * slot_bytes bytes, 256-byte
+ *               aligned, owned by the caller and kept alive until destroy; or
+ *               NULL, in which case the library allocates (and frees) it.
+ *  arena_bytes: size of a caller arena (ignored when arena is NULL).
+ * The library also allocates the slot table (int32 [L][E], every entry -1 =
+ * unmapped), a staging buffer of one slot, a workspace sized from max_tokens
+ * and a device error word.  On failure *out is NULL and nothing is leaked.
+ * Errors: EINVAL (bad config / pointers), ENOMEM, ECUDA.
+ */
+moe_fp4_status moe_fp4_create(const moe_fp4_config *cfg, int device, void *arena,
+                              size_t arena_bytes, moe_fp4_ctx **out);
+
+/* Destroy a context: synchronises the device, frees what the library
+ * allocated.  NULL is ignored. */
+void moe_fp4_destroy(moe_fp4_ctx *ctx);
+
+/* Device pointer to the base of the arena (caller's or the library's). */
+void *moe_fp4_arena(moe_fp4_ctx *ctx);
+
+/* Set an option (MOE_FP4_OPT_PATH, MOE_FP4_OPT_PROFILE).  EINVAL on an
+ * unknown option or value.  With profiling on, route and forward record a
+ * CUDA event pair around each kernel they launch on the caller's stream (this
+ * serialises kernels that would otherwise overlap through programmatic
+ * dependent launch). */
+moe_fp4_status moe_fp4_set_option(moe_fp4_ctx *ctx, int option, int value);
+
+/*
+ * Per-kernel device times of the profiled launches since the last read:
+ * synchronises the device, writes up to `max` records (names[i] points at a
+ * static string such as "gemv_up", ms[i] its event-measured duration in
+ * milliseconds) and returns the number of records (0 when profiling is off),
+ * or -1 on a CUDA error.  Reading clears the record list.
+ */
+int moe_fp4_profile_read(moe_fp4_ctx *ctx, const char **names, float *ms, int max);
+
+/*
+ * Put expert `expert` of layer `layer` into arena slot `slot` and map
+ * (layer, expert) -> slot.  The six tensors are in checkpoint layout
+ * (10100.com article, section "moe专家的容量瓶颈"): w1/w3 codes uint8
+ * [I, H/2] with the even K index in the low nibble, w1/w3 scales UE8M0
+ * [I, H/32], w2 codes [H, I/2], w2 scales [H, I/32].  Each pointer may be
+ * host or device memory (pageable host memory makes the call block until
+ * the copy has been staged).  The copy and re-encode run on `stream`.
+ * Whatever was mapped to `slot` before is unmapped; a previous slot of
+ * (layer, expert) is released.  slot = -1 only unmaps (layer, expert) and the
+ * pointers are ignored.  Supported scale bytes are 2..252 (every value whose
+ * E2M1 multiples are normal bf16 numbers); others latch EINVAL in the error
+ * word.  Errors: EINVAL (indices, NULL tensors), ECUDA.
+ */
+moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx *ctx, int layer, int expert, int slot,
+                                        const uint8_t *w1, const uint8_t *w1_scale,
+                                        const uint8_t *w3, const uint8_t *w3_scale,
+                                        const uint8_t *w2, const uint8_t *w2_scale,
+                                        void *stream);
+
+/*
+ * Route T tokens of one layer (one kernel launch).
+ *  logits    fp32 [T, E], finite (a NaN latches EINVAL).
+ *  keep_mask uint8 [E] or NULL: experts with 0 cannot be chosen (the pruned
+ *            arena of 10100.com, section "方案二", where the router may pick
+ *            only retained experts).  Fewer than k kept experts latches EINVAL.
+ *  ids       int32 [T, k] out: chosen experts, larger logit first, lower index
+ *            first on equal logits (-0.0 == +0.0).
+ *  weights   fp32 [T, k] out: exp(l_j - l_max) / sum over the chosen k.
+ *  counts    int32 [E] out: entries per expert.
+ *  offsets   int32 [E+1] out: exclusive prefix sum of counts.
+ *  perm      int32 [T*k] out: entry indices t*k+j grouped by expert, ascending
+ *            (t, j) inside each expert (a stable counting sort).
+ * `layer` is accepted for symmetry with forward and must be in [0, L).
+ * T = 0 writes zero counts and offsets.  Errors: EINVAL, ECUDA.
+ */
+moe_fp4_status moe_fp4_route(moe_fp4_ctx *ctx, int layer, const float *logits,
+                             const uint8_t *keep_mask, int T, int32_t *ids, float *weights,
+                             int32_t *counts, int32_t *offsets, int32_t *perm, void *stream);
+
+/*
+ * Expert FFN and combine for T tokens of `layer`:
+ *  x         bf16 [T, H] (uint16 bit patterns), 16-byte aligned.
+ *  ids, weights, counts, offsets, perm: as produced by moe_fp4_route.
+ *  y         fp32 [T, H] out, 16-byte aligned:
+ *            sum_j weights[t, j] * expert_{ids[t,j]}(x[t]).
+ *  x_out     bf16 [T, H] out or NULL, 8-byte aligned: bf16_rne(x + y), the
+ *            residual update of a stacked layer; may alias x.
+ * An entry routed to an expert with no slot contributes zero and latches
+ * ESLOT.  Scratch (the bf16 h rows and per-entry fp32 outputs) lives in the
+ * context's workspace, so calls on one context must not overlap in time.
+ * Errors: EINVAL, ECUDA.
+ */
+moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, int T,
+                               const int32_t *ids, const float *weights,
+                               const int32_t *counts, const int32_t *offsets,
+                               const int32_t *perm, float *y, uint16_t *x_out, void *stream);
+
+/*
+ * Synchronise the device, read and clear the device error word.  Returns the
+ * first latched status (OK if none) and writes a one-line description into
+ * msg (n bytes, may be NULL).  Host-side errors of the last failing call are
+ * reported too.
+ */
+moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FP4_H */
