@@ -59,7 +59,10 @@ __device__ __forceinline__ int find_active_expert(const int32_t* offsets, int E,
         bool act = (e < E) && (__ldg(offsets + e + 1) > __ldg(offsets + e));
         uint32_t ball = __ballot_sync(0xFFFFFFFFu, act);
         int cnt = __popc(ball);
-        if (a < cnt) return base + __fns(ball, 0, a + 1);
+        if (a < cnt) {   // warp-uniform: the lane holding the a-th set bit answers
+            uint32_t hit = __ballot_sync(0xFFFFFFFFu, act && __popc(ball & lanemask_lt()) == a);
+            return base + __ffs(hit) - 1;
+        }
         a -= cnt;
     }
     return -1;
@@ -165,8 +168,8 @@ __global__ void __launch_bounds__(NW * 32) gemv_up_kernel(GemvArgs a) {
         red[warp][1][g + 8][2 * c] = d3[2];
         red[warp][1][g + 8][2 * c + 1] = d3[3];
         __syncthreads();
-        if (threadIdx.x < 128) {
-            const int row = threadIdx.x >> 3, tk = threadIdx.x & 7;
+        for (int i = threadIdx.x; i < 128; i += NW * 32) {
+            const int row = i >> 3, tk = i & 7;
             if (tk < ng) {
                 float a1 = 0.f, a3 = 0.f;
 #pragma unroll
@@ -235,8 +238,8 @@ __global__ void __launch_bounds__(NW * 32) gemv_down_kernel(GemvArgs a) {
         red[warp][g + 8][2 * c] = d[2];
         red[warp][g + 8][2 * c + 1] = d[3];
         __syncthreads();
-        if (threadIdx.x < 128) {
-            const int row = threadIdx.x >> 3, tk = threadIdx.x & 7;
+        for (int i = threadIdx.x; i < 128; i += NW * 32) {
+            const int row = i >> 3, tk = i & 7;
             if (tk < ng) {
                 float o = 0.f;
 #pragma unroll
