@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -442,3 +443,105 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx* c, char* msg, size_t n) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward without allocation (moe_fp4_forward_noalloc): the decode kernels
+// with their scratch in a file-scope device array instead of a context
+// workspace.  Host code must not use the array's name as a device address:
+// its device address is looked up once per device with cudaGetSymbolAddress.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(16) << 20;   // 16 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+__device__ int g_noalloc_err_sink[4];                        // errors when err == NULL
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_scratch_dev[kMaxDevices];
+int* g_noalloc_err_dev[kMaxDevices];
+
+// Device addresses of the scratch array and the error sink on the current
+// device (looked up on the first call per device).
+bool noalloc_addresses(int dev, void** scratch, int** sink) {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_scratch_dev[dev]) {
+        void* p = nullptr;
+        void* q = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return false;
+        if (cudaGetSymbolAddress(&q, g_noalloc_err_sink) != cudaSuccess) return false;
+        g_noalloc_err_dev[dev] = static_cast<int*>(q);
+        g_noalloc_scratch_dev[dev] = p;
+    }
+    *scratch = g_noalloc_scratch_dev[dev];
+    *sink = g_noalloc_err_dev[dev];
+    return true;
+}
+
+cudaError_t noalloc_up(int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
+    switch (nw) {
+        case 1: return launch_pdl(gemv_up_kernel<1>, grid, dim3(32), 0, s, a);
+        case 2: return launch_pdl(gemv_up_kernel<2>, grid, dim3(64), 0, s, a);
+        case 4: return launch_pdl(gemv_up_kernel<4>, grid, dim3(128), 0, s, a);
+        case 6: return launch_pdl(gemv_up_kernel<6>, grid, dim3(192), 0, s, a);
+        default: return launch_pdl(gemv_up_kernel<8>, grid, dim3(256), 0, s, a);
+    }
+}
+cudaError_t noalloc_down(int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
+    switch (nw) {
+        case 1: return launch_pdl(gemv_down_kernel<1>, grid, dim3(32), 0, s, a);
+        case 2: return launch_pdl(gemv_down_kernel<2>, grid, dim3(64), 0, s, a);
+        case 4: return launch_pdl(gemv_down_kernel<4>, grid, dim3(128), 0, s, a);
+        case 6: return launch_pdl(gemv_down_kernel<6>, grid, dim3(192), 0, s, a);
+        default: return launch_pdl(gemv_down_kernel<8>, grid, dim3(256), 0, s, a);
+    }
+}
+
+}  // namespace
+
+extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, const uint8_t* arena,
+                                                  const int32_t* slot_table, int layer, const uint16_t* x,
+                                                  int T, const float* weights, const int32_t* offsets,
+                                                  const int32_t* perm, float* y, uint16_t* x_out,
+                                                  int32_t* err, void* stream) {
+    if (!config_ok(cfg) || !arena || !slot_table) return MOE_FP4_EINVAL;
+    if (layer < 0 || layer >= cfg->n_layers || T < 0) return MOE_FP4_EINVAL;
+    if (T == 0) return MOE_FP4_OK;
+    if (!x || !weights || !offsets || !perm || !y) return MOE_FP4_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
+        (reinterpret_cast<uintptr_t>(x_out) & 7) || (reinterpret_cast<uintptr_t>(arena) & 255))
+        return MOE_FP4_EINVAL;
+    const size_t H = cfg->hidden, I = cfg->inter, k = cfg->top_k, E = cfg->n_experts;
+    const size_t ent = static_cast<size_t>(T) * k;
+    const size_t h_bytes = (ent * I * sizeof(uint16_t) + 255) & ~size_t(255);
+    const size_t need = h_bytes + ent * H * sizeof(float);
+    if (need > kNoallocScratchBytes) return MOE_FP4_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_FP4_ECUDA;
+    void* scratch = nullptr;
+    int* sink = nullptr;
+    if (!noalloc_addresses(dev, &scratch, &sink)) return MOE_FP4_ECUDA;
+    uint8_t* sp = static_cast<uint8_t*>(scratch);
+    GemvArgs a{arena, 0, 0, 0, 0, 0, 0, slot_table, layer, static_cast<int>(E), static_cast<int>(k),
+               static_cast<int>(H), static_cast<int>(I), x, offsets, perm,
+               reinterpret_cast<uint16_t*>(sp), reinterpret_cast<float*>(sp + h_bytes),
+               err ? reinterpret_cast<int*>(err) : sink};
+    a.slot_bytes = moe_fp4_slot_bytes(cfg);
+    a.off_w3 = I * H / 2;
+    a.off_w2 = I * H;
+    a.off_s1 = I * H + H * I / 2;
+    a.off_s3 = a.off_s1 + I * H / 32;
+    a.off_s2 = a.off_s3 + I * H / 32;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned active_max = static_cast<unsigned>(ent < E ? ent : E);
+    if (noalloc_up(pick_warps(static_cast<int>(H / 128)), dim3(static_cast<unsigned>(I / 16), active_max), s, a) !=
+            cudaSuccess ||
+        noalloc_down(pick_warps(static_cast<int>(I / 128)), dim3(static_cast<unsigned>(H / 16), active_max), s, a) !=
+            cudaSuccess)
+        return MOE_FP4_ECUDA;
+    const int n4 = T * static_cast<int>(H / 4);
+    if (launch_pdl(combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s, static_cast<const float*>(a.obuf),
+                   weights, x, T, static_cast<int>(H), static_cast<int>(k), y, x_out) != cudaSuccess)
+        return MOE_FP4_ECUDA;
+    return MOE_FP4_OK;
+}

@@ -24,7 +24,7 @@ OPT_PATH, OPT_PROFILE = 1, 2
 # every symbol include/moe_fp4.h declares
 EXPORTS = ("moe_fp4_slot_bytes", "moe_fp4_create", "moe_fp4_destroy", "moe_fp4_arena",
            "moe_fp4_set_option", "moe_fp4_profile_read", "moe_fp4_load_expert_slot", "moe_fp4_route",
-           "moe_fp4_forward", "moe_fp4_last_error")
+           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -71,6 +71,8 @@ def load(path: str = LIB_PATH):
         L.moe_fp4_forward.argtypes = [P, I32, P, I32, P, P, P, P, P, P, P, P]
         L.moe_fp4_last_error.restype = I32
         L.moe_fp4_last_error.argtypes = [P, ctypes.c_char_p, SZ]
+        L.moe_fp4_forward_noalloc.restype = I32
+        L.moe_fp4_forward_noalloc.argtypes = [ctypes.POINTER(Config), P, P, I32, P, I32, P, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -238,3 +240,14 @@ def _data_ptr(t) -> int:
     if isinstance(t, torch.Tensor):
         return t.data_ptr()
     return t.ctypes.data   # numpy array (host memory)
+
+
+def forward_noalloc(cfg: Config, arena_ptr: int, slot_table: torch.Tensor, layer: int, x: torch.Tensor,
+                    r: Routing, y: torch.Tensor, x_out: torch.Tensor | None = None,
+                    err: torch.Tensor | None = None, stream=None) -> int:
+    """moe_fp4_forward_noalloc: the decode forward with library-owned static
+    scratch, for callers that may not allocate device memory.  Returns the
+    status code (EINVAL when T exceeds the scratch limit)."""
+    return load().moe_fp4_forward_noalloc(ctypes.byref(cfg), ctypes.c_void_p(arena_ptr), _ptr(slot_table), layer,
+                                          _ptr(x), x.shape[0], _ptr(r.weights), _ptr(r.offsets), _ptr(r.perm),
+                                          _ptr(y), _ptr(x_out), _ptr(err), _stream(stream))

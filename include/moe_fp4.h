@@ -192,6 +192,49 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, i
  */
 moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
 
+/*
+ * Forward without any allocation: the same decode path as moe_fp4_forward
+ * (grouped GEMV, SwiGLU, combine; always the GEMV kernels), for callers that
+ * cannot call cudaMalloc -- for example a plugin inside a host framework that
+ * owns all device memory and forbids allocation on its execution path, or
+ * code that runs where the CUDA allocator must not be entered.  This call has
+ * no counterpart on the pages: it is a deployment variant of this library.
+ *
+ * Nothing is allocated and no context is used.  The caller passes every input
+ * and output; the two scratch tensors of the forward (bf16 h rows and fp32
+ * per-entry outputs) live in one library-owned, file-scope device array of
+ * 16 MiB (16,777,216 bytes) that every GPU which loads the library holds until
+ * the process exits.  A call needs T*k*(2*I + 4*H) bytes of it (the h part
+ * rounded up to 256); larger T returns EINVAL before any launch.  For the
+ * V4.1 shape that allows T*k <= 668 (T <= 111 at k = 6).
+ *
+ * Every call, on every stream, shares that one array and leaves the last
+ * call's contents in it; nothing in it needs to start at zero.  Calls whose
+ * executions overlap on the GPU race on it: serialise them (one stream, or
+ * events).  The first call on a device looks up the array's device address
+ * with cudaGetSymbolAddress (once per device, that device current); make that
+ * first call before any stream capture.
+ *
+ *  cfg         the layer shape (as for moe_fp4_create; n_slots and max_tokens
+ *              only bound the indices used).
+ *  arena       device, n_slots slots of moe_fp4_slot_bytes(cfg) bytes in the
+ *              library's slot layout (as filled by moe_fp4_load_expert_slot,
+ *              e.g. the arena of a context created elsewhere).
+ *  slot_table  device int32 [n_layers][E]: slot of (layer, expert) or -1.
+ *  x, weights, offsets, perm, y, x_out, T, layer: as for moe_fp4_forward
+ *              (ids and counts are not needed).
+ *  err         device int32 [4] or NULL: first error latched by the kernels
+ *              ([0] status, [1] detail), as moe_fp4_last_error reports them;
+ *              the caller clears it.  With NULL, kernel-found errors are
+ *              dropped.
+ * Errors: EINVAL (arguments, T beyond the scratch limit), ECUDA.
+ */
+moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config *cfg, const uint8_t *arena,
+                                       const int32_t *slot_table, int layer, const uint16_t *x,
+                                       int T, const float *weights, const int32_t *offsets,
+                                       const int32_t *perm, float *y, uint16_t *x_out,
+                                       int32_t *err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
