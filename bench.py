@@ -40,6 +40,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_b1", choices=["decode_b1", "decode_b64", "prefill_2048"])
+    p.add_argument("--experts", type=int, default=0,
+                   help="resident experts override (a smaller arena for ncu captures; 0 = the workload's)")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
     return p.parse_args()
 
@@ -379,6 +381,10 @@ def run_ours(args, wl):
 def main():
     args = parse()
     wl = synth.WORKLOADS[args.workload]
+    if args.experts:
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name}_e{args.experts}", n_experts=args.experts,
+                                 notes=f"{wl.notes} (profiling case: {args.experts} experts)")
     if args.impl == "reference":
         run_reference(args, wl)
     else:

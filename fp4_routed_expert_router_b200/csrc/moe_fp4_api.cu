@@ -15,6 +15,8 @@
 #include "../../include/moe_fp4.h"
 #include "common.cuh"
 #include "decode_gemv.cuh"
+#include "decode_stream.cuh"
+#include "decode_ws.cuh"
 #include "fp4_decode.cuh"
 #include "router.cuh"
 #include "tc_prefill.cuh"
@@ -38,6 +40,7 @@ struct moe_fp4_ctx {
     std::vector<int32_t> h_table;      // host mirror of d_table
     std::vector<int64_t> slot_owner;   // slot -> layer*E+expert or -1
     int path = MOE_FP4_PATH_AUTO;
+    int smem_optin = 0;                // opt-in shared memory per block (bytes)
     bool profile = false;
     struct ProfRec { const char* name; cudaEvent_t a, b; };
     std::vector<ProfRec> prof;         // profiled launches not yet read
@@ -158,6 +161,94 @@ const char* kernel_name(int kid) {
     }
 }
 
+template <bool UP, int NW>
+static cudaError_t launch_stream(moe_fp4_ctx* c, int maxc, dim3 grid, cudaStream_t s, const GemvArgs& a,
+                                 const StreamPlan& p) {
+    const char* name = UP ? "gemv_up" : "gemv_down";
+    const dim3 block(NW * 32);
+    const size_t sm = static_cast<size_t>(p.smem_bytes);
+    switch (maxc) {
+        case 1: return launch_k(c, name, gemv_stream_kernel<UP, NW, 1>, grid, block, sm, s, a, p);
+        case 2: return launch_k(c, name, gemv_stream_kernel<UP, NW, 2>, grid, block, sm, s, a, p);
+        case 3: return launch_k(c, name, gemv_stream_kernel<UP, NW, 3>, grid, block, sm, s, a, p);
+        case 4: return launch_k(c, name, gemv_stream_kernel<UP, NW, 4>, grid, block, sm, s, a, p);
+        case 5: return launch_k(c, name, gemv_stream_kernel<UP, NW, 5>, grid, block, sm, s, a, p);
+        default: return launch_k(c, name, gemv_stream_kernel<UP, NW, 8>, grid, block, sm, s, a, p);
+    }
+}
+
+template <bool UP, int NW>
+static cudaError_t allow_stream_smem(int bytes) {
+    cudaError_t e = cudaSuccess;
+    auto set = [&](const void* f) {
+        cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (r != cudaSuccess) e = r;
+    };
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 1>));
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 2>));
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 3>));
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 4>));
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 5>));
+    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 8>));
+    return e;
+}
+
+constexpr int kUpWarps = 8, kDownWarps = 6;
+
+static int stream_maxc(int nchunks, int nw) {
+    const int m = (nchunks + nw - 1) / nw;
+    return m <= 5 ? m : (m <= 8 ? 8 : 0);   // 0: shape not covered by the stream kernels
+}
+
+// Grouped GEMV decode through the streaming kernels; false when the shape
+// needs the plain kernels instead.
+static bool stream_decode(moe_fp4_ctx* c, const GemvArgs& a, int active_max, cudaStream_t s, cudaError_t* err) {
+    const int H = a.H, I = a.I;
+    const int mu = stream_maxc(H / 128, kUpWarps), md = stream_maxc(I / 128, kDownWarps);
+    if (!mu || !md || c->smem_optin <= 0) return false;
+    const StreamPlan pu = make_stream_plan(true, H, I, a.E, active_max, kUpWarps, c->smem_optin);
+    const StreamPlan pd = make_stream_plan(false, H, I, a.E, active_max, kDownWarps, c->smem_optin);
+    if (!pu.stages || !pd.stages) return false;
+    const int tu = active_max * (I / 16), td = active_max * (H / 16);
+    const dim3 gu(static_cast<unsigned>(tu < c->sm_count ? tu : c->sm_count));
+    const dim3 gd(static_cast<unsigned>(td < c->sm_count ? td : c->sm_count));
+    *err = launch_stream<true, kUpWarps>(c, mu, gu, s, a, pu);
+    if (*err == cudaSuccess) *err = launch_stream<false, kDownWarps>(c, md, gd, s, a, pd);
+    return true;
+}
+
+// ---- warp-specialised decode GEMV (the default decode path)
+template <bool UP, int RB, int KS, int CPW>
+cudaError_t launch_ws(moe_fp4_ctx* c, dim3 grid, cudaStream_t s, const GemvArgs& a, const WsPlan& p) {
+    return launch_k(c, UP ? "gemv_up" : "gemv_down", gemv_ws_kernel<UP, RB, KS, CPW>, grid,
+                    dim3((RB * KS + 1) * 32), static_cast<size_t>(p.smem_bytes), s, a, p);
+}
+
+template <bool UP, int RB, int KS, int CPW>
+cudaError_t allow_ws_smem(int bytes) {
+    return cudaFuncSetAttribute(reinterpret_cast<const void*>(gemv_ws_kernel<UP, RB, KS, CPW>),
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Shapes with a warp-specialised instantiation: (K chunks of 128) -> (KS, CPW).
+//   up:   40 chunks (H 5120) -> 10 x 4;  2 chunks (H 256) -> 2 x 1;  RB 1
+//   down: 18 chunks (I 2304) ->  9 x 2;  1 chunk  (I 128) -> 1 x 1;  RB 2
+bool ws_decode(moe_fp4_ctx* c, const GemvArgs& a, int active_max, cudaStream_t s, cudaError_t* err) {
+    const int H = a.H, I = a.I, cu = H / 128, cd = I / 128;
+    if (c->smem_optin <= 0 || H % 32 || !((cu == 40 || cu == 2) && (cd == 18 || cd == 1))) return false;
+    const int ncu = cu == 40 ? 10 : 2, ncd = cd == 18 ? 18 : 2;
+    const WsPlan pu = make_ws_plan(true, H, I, a.E, active_max, 1, ncu, c->smem_optin);
+    const WsPlan pd = make_ws_plan(false, H, I, a.E, active_max, 2, ncd, c->smem_optin);
+    if (!pu.stages || !pd.stages) return false;
+    const int tu = active_max * (I / 16), td = active_max * (H / 32);
+    const dim3 gu(static_cast<unsigned>(tu < c->sm_count ? tu : c->sm_count));
+    const dim3 gd(static_cast<unsigned>(td < c->sm_count ? td : c->sm_count));
+    *err = (cu == 40) ? launch_ws<true, 1, 10, 4>(c, gu, s, a, pu) : launch_ws<true, 1, 2, 1>(c, gu, s, a, pu);
+    if (*err != cudaSuccess) return true;
+    *err = (cd == 18) ? launch_ws<false, 2, 9, 2>(c, gd, s, a, pd) : launch_ws<false, 2, 1, 1>(c, gd, s, a, pd);
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -194,6 +285,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     int major = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
     cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
+    cudaDeviceGetAttribute(&c->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     if (major < 10) return bail(MOE_FP4_ECUDA);   // sm_100a code only
     if (arena) {
         c->arena = static_cast<uint8_t*>(arena);
@@ -212,6 +304,16 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         return bail(MOE_FP4_ENOMEM);
     }
     if (tc_plan_create(&c->tc, *cfg) != cudaSuccess) { cudaGetLastError(); return bail(MOE_FP4_ENOMEM); }
+    c->smem_optin -= 1024;   // room for the kernels' static shared memory
+    if (allow_stream_smem<true, kUpWarps>(c->smem_optin) != cudaSuccess ||
+        allow_stream_smem<false, kDownWarps>(c->smem_optin) != cudaSuccess ||
+        allow_ws_smem<true, 1, 10, 4>(c->smem_optin) != cudaSuccess ||
+        allow_ws_smem<true, 1, 2, 1>(c->smem_optin) != cudaSuccess ||
+        allow_ws_smem<false, 2, 9, 2>(c->smem_optin) != cudaSuccess ||
+        allow_ws_smem<false, 2, 1, 1>(c->smem_optin) != cudaSuccess) {
+        cudaGetLastError();
+        c->smem_optin = 0;   // the plain kernels need no opt-in
+    }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
         cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
@@ -318,7 +420,14 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx* c, int layer, const float* logits, con
     const size_t smem = sizeof(int) * kRouteWarps * g.n_experts;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (g.n_experts <= 128)
+    if (T * g.top_k <= 32) {   // one warp: route + bitonic grouping
+        if (g.n_experts <= 128)
+            e = launch_k(c, "route", route_small_kernel<4>, dim3(1), dim3(32), 0, s, a);
+        else if (g.n_experts <= 384)
+            e = launch_k(c, "route", route_small_kernel<12>, dim3(1), dim3(32), 0, s, a);
+        else
+            e = launch_k(c, "route", route_small_kernel<32>, dim3(1), dim3(32), 0, s, a);
+    } else if (g.n_experts <= 128)
         e = launch_k(c, "route", route_kernel<4>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
     else if (g.n_experts <= 384)
         e = launch_k(c, "route", route_kernel<12>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
@@ -378,6 +487,10 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     if (use_tc) {
         e = tc_forward(&c->tc, a, T, s);
         if (e != cudaSuccess) return cuda_fail(c, e, "forward: tc launch");
+    } else if (ws_decode(c, a, active_max, s, &e)) {
+        if (e != cudaSuccess) return cuda_fail(c, e, "forward: decode launch");
+    } else if (stream_decode(c, a, active_max, s, &e)) {
+        if (e != cudaSuccess) return cuda_fail(c, e, "forward: stream launch");
     } else {
         e = launch_up(c, pick_warps(H / 128), dim3(I / 16, active_max), s, a);
         if (e != cudaSuccess) return cuda_fail(c, e, "forward: up launch");

@@ -173,6 +173,12 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kRouteWarps + warp;
     if (t < a.T) route_token<NI>(a, t, lane);
+    if (gridDim.x == 1) {        // the only CTA: no ticket needed
+        __syncthreads();
+        group_entries(a, smem_hist);
+        pdl_trigger();
+        return;
+    }
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -186,6 +192,67 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     group_entries(a, smem_hist);
     pdl_trigger();
     if (threadIdx.x == 0) *a.ticket = 0;
+}
+
+
+// ---------------------------------------------------------------------------
+// Small batches (T*k <= 32): one warp routes the tokens, then groups the
+// entries with a 32-lane bitonic sort on (expert, entry) keys; per-expert
+// offsets come from binary searches in the sorted experts.  No grid-wide
+// ticket, fence or CTA barrier on the critical path.
+template <int NI>
+__global__ void __launch_bounds__(32) route_small_kernel(RouteArgs a) {
+    pdl_wait();
+    const int lane = threadIdx.x;
+    const int n = a.T * a.k;            // <= 32
+    uint32_t key = 0xFFFFFFFFu;         // (expert << 5) | entry; empty lanes sort last
+    for (int t = 0; t < a.T; ++t) {
+        route_token<NI>(a, t, lane);
+        // the chosen experts were just written by lanes 0..k-1 of this warp
+        __syncwarp();
+        const int q = lane - t * a.k;
+        if (q >= 0 && q < a.k) {
+            const int e = a.ids[static_cast<size_t>(t) * a.k + q];
+            key = (static_cast<uint32_t>(e) << 5) | static_cast<uint32_t>(lane);
+        }
+    }
+    // bitonic sort of 32 keys across the warp, ascending
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, key, stride);
+            const bool ascending = ((lane & size) == 0);
+            const bool lower = ((lane & stride) == 0);
+            const uint32_t lo = min(key, other), hi = max(key, other);
+            key = (lower == ascending) ? lo : hi;
+        }
+    }
+    pdl_trigger();
+    if (lane < n) a.perm[lane] = static_cast<int32_t>(key & 31u);
+    const int sorted_e = (lane < n) ? static_cast<int>(key >> 5) : 0x7FFFFFFF;
+    // lower_bound(e) = #entries with expert < e, by a branch-free binary search
+    // over the sorted experts held one per lane (all lanes shuffle together)
+    auto lower_bound = [&](int e) {
+        int pos = 0;
+#pragma unroll
+        for (int step = 16; step > 0; step >>= 1) {
+            const int v = __shfl_sync(0xFFFFFFFFu, sorted_e, pos + step - 1);
+            if (v < e) pos += step;
+        }
+        const int v = __shfl_sync(0xFFFFFFFFu, sorted_e, pos & 31);
+        return (pos < 32 && v < e) ? pos + 1 : pos;
+    };
+    for (int base = 0; base <= a.E; base += 32) {
+        const int e = base + lane;
+        const int lb0 = lower_bound(e), lb1 = lower_bound(e + 1);
+        if (e < a.E) {
+            a.offsets[e] = lb0;
+            a.counts[e] = lb1 - lb0;
+        } else if (e == a.E) {
+            a.offsets[e] = n;
+        }
+    }
 }
 
 }  // namespace moe

@@ -52,10 +52,11 @@ def test_tiny_zero_tokens(tiny):
     assert int(r.counts.sum()) == 0 and int(r.offsets[-1]) == 0
 
 
-def test_tiny_routing_ties_and_mask(tiny):
+@pytest.mark.parametrize("T", [5, 16, 40])   # one-warp path (T*k <= 32) and the grid path
+def test_tiny_routing_ties_and_mask(tiny, T):
     wl = tiny.wl
-    rng = np.random.default_rng(5)
-    logits = rng.integers(-2, 3, size=(40, wl.n_experts)).astype(np.float32)
+    rng = np.random.default_rng(5 + T)
+    logits = rng.integers(-2, 3, size=(T, wl.n_experts)).astype(np.float32)
     logits[0, 3] = -0.0
     logits[0, 1] = 0.0
     keep = np.ones(wl.n_experts, np.uint8)
