@@ -76,11 +76,15 @@ __host__ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t y, u
 // (k6,k7), lower K index in the low half.
 __host__ __device__ __forceinline__ void fp4_decode8(uint32_t w, const Fp4Lut& t, uint32_t out[4]) {
     uint32_t m = w & 0x77777777u;
+#ifdef __CUDA_ARCH__
+    uint32_t mb = __umulhi(m, 0x10000u);     // m >> 16 on the multiply pipe
+#else
     uint32_t mb = m >> 16;
+#endif
     uint32_t loA = byte_perm(t.l0, t.l1, m);
     uint32_t hiA = byte_perm(t.h0, t.h1, m) | (w & 0x80808080u);
     uint32_t loB = byte_perm(t.l0, t.l1, mb);
-    uint32_t hiB = byte_perm(t.h0, t.h1, mb) | ((w << 4) & 0x80808080u);
+    uint32_t hiB = byte_perm(t.h0, t.h1, mb) | ((w * 16u) & 0x80808080u);
     out[0] = byte_perm(loA, hiA, 0x5140);
     out[1] = byte_perm(loA, hiA, 0x7362);
     out[2] = byte_perm(loB, hiB, 0x5140);

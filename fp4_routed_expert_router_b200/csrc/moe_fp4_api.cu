@@ -14,11 +14,11 @@
 
 #include "../../include/moe_fp4.h"
 #include "common.cuh"
-#include "decode_gemv.cuh"
-#include "decode_stream.cuh"
-#include "decode_ws.cuh"
+#include "decode_common.cuh"
+#include "decode_tile.cuh"
 #include "fp4_decode.cuh"
 #include "router.cuh"
+#include "slot_layout.cuh"
 #include "tc_prefill.cuh"
 
 using namespace moe;
@@ -28,7 +28,7 @@ struct moe_fp4_ctx {
     int device = 0;
     int sm_count = 0;
     size_t slot_bytes = 0;
-    size_t off_w3 = 0, off_w2 = 0, off_s1 = 0, off_s3 = 0, off_s2 = 0;
+    SlotLayout lay{};                  // arrangement of an expert inside its slot
     uint8_t* arena = nullptr;
     bool own_arena = false;
     int32_t* d_table = nullptr;        // [L][E]
@@ -125,26 +125,64 @@ cudaError_t launch_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim
     return e;
 }
 
-// Re-encode the code words of one expert (staging, checkpoint layout) into
-// its slot, copy the scales, check every scale byte is in [2, 252], and map
-// the slot.  One thread per 32-bit word of codes / per 4 scale bytes.
-__global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
-                                 size_t code_words, size_t scale_bytes, int32_t* table,
-                                 int map_index, int slot, int* err) {
+// Re-lay one expert from the staging buffer (checkpoint layout: w1, w3, w2
+// codes, then s1, s3, s2 scales, row-major) into its slot (slot_layout.cuh):
+// one thread per 16-byte chunk of codes (re-encoded, placed in its block at
+// its swizzled position) and one thread per scale byte (checked against the
+// supported range [2, 252]).  Thread 0 maps (layer, expert) -> slot.
+__global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, SlotLayout L,
+                                 int32_t* table, int map_index, int slot, int* err) {
+    const size_t H = L.H, I = L.I, KBu = L.KBu, nfu = L.nfu, KBd = L.KBd, nfd = L.nfd;
+    const size_t n13 = I * H / 32, n2 = H * I / 32;        // 16-byte code chunks of w1 (w3), w2
+    const size_t s13 = I * H / 32, s2 = H * I / 32;        // scale bytes of s1 (s3), s2
     const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
-    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src);
-    uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
-    if (i < code_words) {
-        d32[i] = fp4_reencode_word(s32[i]);
-    } else if (i < code_words + (scale_bytes + 3) / 4) {
-        const size_t b0 = (i - code_words) * 4;
-        for (size_t b = b0; b < b0 + 4 && b < scale_bytes; ++b) {
-            const uint8_t v = src[code_words * 4 + b];
-            dst[code_words * 4 + b] = v;
-            if (v < 2 || v > 252) latch_error(err, ERR_EINVAL, static_cast<int>(b), KID_LOAD);
-        }
-    }
     if (i == 0 && map_index >= 0) table[map_index] = slot;
+    if (i < 2 * n13 + n2) {
+        size_t so, dofs;
+        if (i < 2 * n13) {                                   // w1 / w3 chunk
+            const size_t mat = i / n13, rem = i - mat * n13;
+            const size_t r = rem / (H / 32), q = rem - r * (H / 32);
+            const size_t f = q / (KBu / 32), qi = q - f * (KBu / 32);
+            so = mat * (I * H / 2) + r * (H / 2) + q * 16;
+            dofs = ((r / 16) * nfu + f) * L.UB + mat * 16 * (KBu / 2) + (r % 16) * (KBu / 2) +
+                   static_cast<size_t>(swizzle_chunk(static_cast<int>(qi), static_cast<int>(r % 16),
+                                                     static_cast<int>(KBu / 2))) * 16;
+        } else {                                             // w2 chunk
+            const size_t rem = i - 2 * n13;
+            const size_t r = rem / (I / 32), q = rem - r * (I / 32);
+            const size_t f = q / (KBd / 32), qi = q - f * (KBd / 32);
+            so = I * H + r * (I / 2) + q * 16;
+            dofs = L.up_bytes + ((r / 16) * nfd + f) * L.DB + (r % 16) * (KBd / 2) +
+                   static_cast<size_t>(swizzle_chunk(static_cast<int>(qi), static_cast<int>(r % 16),
+                                                     static_cast<int>(KBd / 2))) * 16;
+        }
+        const uint4 v = *reinterpret_cast<const uint4*>(src + so);
+        uint4 w;
+        w.x = fp4_reencode_word(v.x);
+        w.y = fp4_reencode_word(v.y);
+        w.z = fp4_reencode_word(v.z);
+        w.w = fp4_reencode_word(v.w);
+        *reinterpret_cast<uint4*>(dst + dofs) = w;
+        return;
+    }
+    const size_t b = i - (2 * n13 + n2);
+    if (b >= 2 * s13 + s2) return;
+    const size_t sbase = 3 * I * H / 2;                      // scales start after the codes
+    size_t dofs;
+    if (b < 2 * s13) {                                       // s1 / s3 byte
+        const size_t mat = b / s13, rem = b - mat * s13;
+        const size_t r = rem / (H / 32), q = rem - r * (H / 32);
+        const size_t f = q / (KBu / 32), qi = q - f * (KBu / 32);
+        dofs = ((r / 16) * nfu + f) * L.UB + 32 * (KBu / 2) + mat * 16 * (KBu / 32) + (r % 16) * (KBu / 32) + qi;
+    } else {                                                 // s2 byte
+        const size_t rem = b - 2 * s13;
+        const size_t r = rem / (I / 32), q = rem - r * (I / 32);
+        const size_t f = q / (KBd / 32), qi = q - f * (KBd / 32);
+        dofs = L.up_bytes + ((r / 16) * nfd + f) * L.DB + 16 * (KBd / 2) + (r % 16) * (KBd / 32) + qi;
+    }
+    const uint8_t v = src[sbase + b];
+    dst[dofs] = v;
+    if (v < 2 || v > 252) latch_error(err, ERR_EINVAL, static_cast<int>(b), KID_LOAD);
 }
 
 const char* kernel_name(int kid) {
@@ -161,92 +199,54 @@ const char* kernel_name(int kid) {
     }
 }
 
-template <bool UP, int NW>
-static cudaError_t launch_stream(moe_fp4_ctx* c, int maxc, dim3 grid, cudaStream_t s, const GemvArgs& a,
-                                 const StreamPlan& p) {
-    const char* name = UP ? "gemv_up" : "gemv_down";
-    const dim3 block(NW * 32);
-    const size_t sm = static_cast<size_t>(p.smem_bytes);
-    switch (maxc) {
-        case 1: return launch_k(c, name, gemv_stream_kernel<UP, NW, 1>, grid, block, sm, s, a, p);
-        case 2: return launch_k(c, name, gemv_stream_kernel<UP, NW, 2>, grid, block, sm, s, a, p);
-        case 3: return launch_k(c, name, gemv_stream_kernel<UP, NW, 3>, grid, block, sm, s, a, p);
-        case 4: return launch_k(c, name, gemv_stream_kernel<UP, NW, 4>, grid, block, sm, s, a, p);
-        case 5: return launch_k(c, name, gemv_stream_kernel<UP, NW, 5>, grid, block, sm, s, a, p);
-        default: return launch_k(c, name, gemv_stream_kernel<UP, NW, 8>, grid, block, sm, s, a, p);
-    }
-}
-
-template <bool UP, int NW>
-static cudaError_t allow_stream_smem(int bytes) {
-    cudaError_t e = cudaSuccess;
-    auto set = [&](const void* f) {
-        cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (r != cudaSuccess) e = r;
-    };
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 1>));
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 2>));
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 3>));
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 4>));
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 5>));
-    set(reinterpret_cast<const void*>(gemv_stream_kernel<UP, NW, 8>));
-    return e;
-}
-
-constexpr int kUpWarps = 8, kDownWarps = 6;
-
-static int stream_maxc(int nchunks, int nw) {
-    const int m = (nchunks + nw - 1) / nw;
-    return m <= 5 ? m : (m <= 8 ? 8 : 0);   // 0: shape not covered by the stream kernels
-}
-
-// Grouped GEMV decode through the streaming kernels; false when the shape
-// needs the plain kernels instead.
-static bool stream_decode(moe_fp4_ctx* c, const GemvArgs& a, int active_max, cudaStream_t s, cudaError_t* err) {
-    const int H = a.H, I = a.I;
-    const int mu = stream_maxc(H / 128, kUpWarps), md = stream_maxc(I / 128, kDownWarps);
-    if (!mu || !md || c->smem_optin <= 0) return false;
-    const StreamPlan pu = make_stream_plan(true, H, I, a.E, active_max, kUpWarps, c->smem_optin);
-    const StreamPlan pd = make_stream_plan(false, H, I, a.E, active_max, kDownWarps, c->smem_optin);
-    if (!pu.stages || !pd.stages) return false;
-    const int tu = active_max * (I / 16), td = active_max * (H / 16);
-    const dim3 gu(static_cast<unsigned>(tu < c->sm_count ? tu : c->sm_count));
-    const dim3 gd(static_cast<unsigned>(td < c->sm_count ? td : c->sm_count));
-    *err = launch_stream<true, kUpWarps>(c, mu, gu, s, a, pu);
-    if (*err == cudaSuccess) *err = launch_stream<false, kDownWarps>(c, md, gd, s, a, pd);
-    return true;
-}
-
-// ---- warp-specialised decode GEMV (the default decode path)
+// ---- decode path: the tile-streaming GEMV kernels (decode_tile.cuh)
+// Instantiated shapes (RB, KS, CPW):
+//   up   RB 1: 40 chunks (H 5120) -> KS 10 x CPW 4; 2 chunks (H 256) -> 2 x 1
+//   down RB 2: 18 chunks (I 2304) -> KS  9 x CPW 2; 1 chunk  (I 128) -> 1 x 1
 template <bool UP, int RB, int KS, int CPW>
-cudaError_t launch_ws(moe_fp4_ctx* c, dim3 grid, cudaStream_t s, const GemvArgs& a, const WsPlan& p) {
-    return launch_k(c, UP ? "gemv_up" : "gemv_down", gemv_ws_kernel<UP, RB, KS, CPW>, grid,
-                    dim3((RB * KS + 1) * 32), static_cast<size_t>(p.smem_bytes), s, a, p);
+cudaError_t launch_tile(moe_fp4_ctx* c, dim3 grid, cudaStream_t s, const GemvArgs& a, const SlotLayout& L,
+                        const TilePlan& p) {
+    const dim3 block((RB * KS + 1) * 32);
+    if (c) return launch_k(c, UP ? "gemv_up" : "gemv_down", gemv_tile_kernel<UP, RB, KS, CPW>, grid, block,
+                           static_cast<size_t>(p.smem_bytes), s, a, L, p);
+    return launch_pdl(gemv_tile_kernel<UP, RB, KS, CPW>, grid, block, static_cast<size_t>(p.smem_bytes), s, a, L, p);
 }
 
 template <bool UP, int RB, int KS, int CPW>
-cudaError_t allow_ws_smem(int bytes) {
-    return cudaFuncSetAttribute(reinterpret_cast<const void*>(gemv_ws_kernel<UP, RB, KS, CPW>),
+cudaError_t allow_tile_smem(int bytes) {
+    return cudaFuncSetAttribute(reinterpret_cast<const void*>(gemv_tile_kernel<UP, RB, KS, CPW>),
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-// Shapes with a warp-specialised instantiation: (K chunks of 128) -> (KS, CPW).
-//   up:   40 chunks (H 5120) -> 10 x 4;  2 chunks (H 256) -> 2 x 1;  RB 1
-//   down: 18 chunks (I 2304) ->  9 x 2;  1 chunk  (I 128) -> 1 x 1;  RB 2
-bool ws_decode(moe_fp4_ctx* c, const GemvArgs& a, int active_max, cudaStream_t s, cudaError_t* err) {
-    const int H = a.H, I = a.I, cu = H / 128, cd = I / 128;
-    if (c->smem_optin <= 0 || H % 32 || !((cu == 40 || cu == 2) && (cd == 18 || cd == 1))) return false;
-    const int ncu = cu == 40 ? 10 : 2, ncd = cd == 18 ? 18 : 2;
-    const WsPlan pu = make_ws_plan(true, H, I, a.E, active_max, 1, ncu, c->smem_optin);
-    const WsPlan pd = make_ws_plan(false, H, I, a.E, active_max, 2, ncd, c->smem_optin);
-    if (!pu.stages || !pd.stages) return false;
-    const int tu = active_max * (I / 16), td = active_max * (H / 32);
-    const dim3 gu(static_cast<unsigned>(tu < c->sm_count ? tu : c->sm_count));
-    const dim3 gd(static_cast<unsigned>(td < c->sm_count ? td : c->sm_count));
-    *err = (cu == 40) ? launch_ws<true, 1, 10, 4>(c, gu, s, a, pu) : launch_ws<true, 1, 2, 1>(c, gu, s, a, pu);
-    if (*err != cudaSuccess) return true;
-    *err = (cd == 18) ? launch_ws<false, 2, 9, 2>(c, gd, s, a, pd) : launch_ws<false, 2, 1, 1>(c, gd, s, a, pd);
-    return true;
+bool decode_shape_ok(const SlotLayout& L) {
+    const int cu = L.H / 128, cd = L.I / 128;
+    return (cu == 40 || cu == 2) && (cd == 18 || cd == 1) && L.H % 32 == 0;
+}
+
+cudaError_t allow_decode_smem_all(int bytes) {
+    cudaError_t e = cudaSuccess, r;
+    if ((r = allow_tile_smem<true, 1, 10, 4>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_tile_smem<true, 1, 2, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_tile_smem<false, 2, 9, 2>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_tile_smem<false, 2, 1, 1>(bytes)) != cudaSuccess) e = r;
+    return e;
+}
+
+// Launch up then down (c may be NULL: no profiling).  smem_limit: opt-in
+// shared memory per block minus the kernels' static shared memory.
+cudaError_t decode_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& L, int active_max, int sm_count,
+                           int smem_limit, cudaStream_t s) {
+    if (!decode_shape_ok(L)) return cudaErrorNotSupported;
+    const bool big_up = (L.H / 128 == 40), big_down = (L.I / 128 == 18);
+    const TilePlan pu = make_tile_plan(true, L, 1, big_up ? 10 : 2, a.E, active_max, smem_limit);
+    const TilePlan pd = make_tile_plan(false, L, 2, big_down ? 18 : 2, a.E, active_max, smem_limit);
+    if (!pu.stages || !pd.stages) return cudaErrorNotSupported;
+    const dim3 grid(static_cast<unsigned>(sm_count));
+    cudaError_t e = big_up ? launch_tile<true, 1, 10, 4>(c, grid, s, a, L, pu)
+                           : launch_tile<true, 1, 2, 1>(c, grid, s, a, L, pu);
+    if (e != cudaSuccess) return e;
+    return big_down ? launch_tile<false, 2, 9, 2>(c, grid, s, a, L, pd)
+                    : launch_tile<false, 2, 1, 1>(c, grid, s, a, L, pd);
 }
 
 }  // namespace
@@ -269,11 +269,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     c->device = device;
     const size_t H = cfg->hidden, I = cfg->inter, E = cfg->n_experts, L = cfg->n_layers;
     c->slot_bytes = moe_fp4_slot_bytes(cfg);
-    c->off_w3 = I * H / 2;
-    c->off_w2 = I * H;
-    c->off_s1 = I * H + H * I / 2;
-    c->off_s3 = c->off_s1 + I * H / 32;
-    c->off_s2 = c->off_s3 + I * H / 32;
+    c->lay = make_slot_layout(cfg->hidden, cfg->inter);
     const size_t need = c->slot_bytes * static_cast<size_t>(cfg->n_slots);
     auto bail = [&](moe_fp4_status s) {
         moe_fp4_destroy(c);
@@ -305,14 +301,9 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     }
     if (tc_plan_create(&c->tc, *cfg) != cudaSuccess) { cudaGetLastError(); return bail(MOE_FP4_ENOMEM); }
     c->smem_optin -= 1024;   // room for the kernels' static shared memory
-    if (allow_stream_smem<true, kUpWarps>(c->smem_optin) != cudaSuccess ||
-        allow_stream_smem<false, kDownWarps>(c->smem_optin) != cudaSuccess ||
-        allow_ws_smem<true, 1, 10, 4>(c->smem_optin) != cudaSuccess ||
-        allow_ws_smem<true, 1, 2, 1>(c->smem_optin) != cudaSuccess ||
-        allow_ws_smem<false, 2, 9, 2>(c->smem_optin) != cudaSuccess ||
-        allow_ws_smem<false, 2, 1, 1>(c->smem_optin) != cudaSuccess) {
+    if (allow_decode_smem_all(c->smem_optin) != cudaSuccess) {
         cudaGetLastError();
-        c->smem_optin = 0;   // the plain kernels need no opt-in
+        return bail(MOE_FP4_ECUDA);
     }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
@@ -386,18 +377,19 @@ moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx* c, int layer, int expert, i
         if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: evict");
     }
     const size_t H = g.hidden, I = g.inter;
+    const size_t c13 = I * H / 2, sc0 = 3 * I * H / 2;     // checkpoint layout in the staging buffer
     const struct { const uint8_t* p; size_t off, n; } parts[6] = {
-        {w1, 0, I * H / 2},          {w3, c->off_w3, I * H / 2},       {w2, c->off_w2, H * I / 2},
-        {w1_scale, c->off_s1, I * H / 32}, {w3_scale, c->off_s3, I * H / 32}, {w2_scale, c->off_s2, H * I / 32}};
+        {w1, 0, c13},           {w3, c13, c13},                 {w2, 2 * c13, H * I / 2},
+        {w1_scale, sc0, I * H / 32}, {w3_scale, sc0 + I * H / 32, I * H / 32},
+        {w2_scale, sc0 + 2 * I * H / 32, H * I / 32}};
     for (const auto& p : parts) {
         e = cudaMemcpyAsync(c->d_staging + p.off, p.p, p.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: copy");
     }
-    const size_t code_words = c->off_s1 / 4, scale_bytes = c->slot_bytes - c->off_s1;
-    const size_t threads = code_words + (scale_bytes + 3) / 4;
+    const size_t threads = 3 * I * H / 32 + 3 * I * H / 32;  // code chunks + scale bytes
     load_slot_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-        c->d_staging, c->arena + static_cast<size_t>(slot) * c->slot_bytes, code_words, scale_bytes,
-        c->d_table, idx, slot, c->d_err);
+        c->d_staging, c->arena + static_cast<size_t>(slot) * c->slot_bytes, c->lay, c->d_table, idx, slot,
+        c->d_err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: launch");
     c->h_table[idx] = slot;
@@ -436,31 +428,6 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx* c, int layer, const float* logits, con
     return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "route: launch");
 }
 
-static int pick_warps(int nchunks) {
-    for (int w : {8, 6, 4, 2, 1})
-        if (nchunks % w == 0) return w;
-    return 8;
-}
-
-static cudaError_t launch_up(moe_fp4_ctx* c, int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
-    switch (nw) {
-        case 1: return launch_k(c, "gemv_up", gemv_up_kernel<1>, grid, dim3(32), 0, s, a);
-        case 2: return launch_k(c, "gemv_up", gemv_up_kernel<2>, grid, dim3(64), 0, s, a);
-        case 4: return launch_k(c, "gemv_up", gemv_up_kernel<4>, grid, dim3(128), 0, s, a);
-        case 6: return launch_k(c, "gemv_up", gemv_up_kernel<6>, grid, dim3(192), 0, s, a);
-        default: return launch_k(c, "gemv_up", gemv_up_kernel<8>, grid, dim3(256), 0, s, a);
-    }
-}
-static cudaError_t launch_down(moe_fp4_ctx* c, int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
-    switch (nw) {
-        case 1: return launch_k(c, "gemv_down", gemv_down_kernel<1>, grid, dim3(32), 0, s, a);
-        case 2: return launch_k(c, "gemv_down", gemv_down_kernel<2>, grid, dim3(64), 0, s, a);
-        case 4: return launch_k(c, "gemv_down", gemv_down_kernel<4>, grid, dim3(128), 0, s, a);
-        case 6: return launch_k(c, "gemv_down", gemv_down_kernel<6>, grid, dim3(192), 0, s, a);
-        default: return launch_k(c, "gemv_down", gemv_down_kernel<8>, grid, dim3(256), 0, s, a);
-    }
-}
-
 moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int T, const int32_t* ids,
                                const float* weights, const int32_t* counts, const int32_t* offsets,
                                const int32_t* perm, float* y, uint16_t* x_out, void* stream) {
@@ -480,23 +447,11 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     const int H = g.hidden, I = g.inter, E = g.n_experts, k = g.top_k;
     const int ent = T * k;
     const int active_max = ent < E ? ent : E;
-    GemvArgs a{c->arena, c->slot_bytes, c->off_w3, c->off_w2, c->off_s1, c->off_s3, c->off_s2,
-               c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_h, c->d_o, c->d_err};
-    bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
-    cudaError_t e;
-    if (use_tc) {
-        e = tc_forward(&c->tc, a, T, s);
-        if (e != cudaSuccess) return cuda_fail(c, e, "forward: tc launch");
-    } else if (ws_decode(c, a, active_max, s, &e)) {
-        if (e != cudaSuccess) return cuda_fail(c, e, "forward: decode launch");
-    } else if (stream_decode(c, a, active_max, s, &e)) {
-        if (e != cudaSuccess) return cuda_fail(c, e, "forward: stream launch");
-    } else {
-        e = launch_up(c, pick_warps(H / 128), dim3(I / 16, active_max), s, a);
-        if (e != cudaSuccess) return cuda_fail(c, e, "forward: up launch");
-        e = launch_down(c, pick_warps(I / 128), dim3(H / 16, active_max), s, a);
-        if (e != cudaSuccess) return cuda_fail(c, e, "forward: down launch");
-    }
+    GemvArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_h, c->d_o, c->d_err};
+    const bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
+    cudaError_t e = use_tc ? tc_forward(&c->tc, a, T, s)
+                           : decode_forward(c, a, c->lay, active_max, c->sm_count, c->smem_optin, s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "forward: expert FFN launch");
     const int n4 = T * (H / 4);
     e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
                  static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
@@ -570,44 +525,41 @@ __device__ int g_noalloc_err_sink[4];                        // errors when err 
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_scratch_dev[kMaxDevices];
-int* g_noalloc_err_dev[kMaxDevices];
 
 // Device addresses of the scratch array and the error sink on the current
 // device (looked up on the first call per device).
-bool noalloc_addresses(int dev, void** scratch, int** sink) {
+// Per-device set-up on the first call (that device current): the device
+// addresses of the scratch array and of the error sink, the SM count, the
+// opt-in shared memory, and the kernels' shared-memory attribute.
+struct NoallocDevice {
+    void* scratch;
+    int* sink;
+    int sm_count;
+    int smem_limit;
+};
+NoallocDevice g_noalloc_dev[kMaxDevices];
+
+bool noalloc_setup(int dev, NoallocDevice* out) {
     if (dev < 0 || dev >= kMaxDevices) return false;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_scratch_dev[dev]) {
+    NoallocDevice& d = g_noalloc_dev[dev];
+    if (!d.scratch) {
         void* p = nullptr;
         void* q = nullptr;
+        int sms = 0, optin = 0;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return false;
         if (cudaGetSymbolAddress(&q, g_noalloc_err_sink) != cudaSuccess) return false;
-        g_noalloc_err_dev[dev] = static_cast<int*>(q);
-        g_noalloc_scratch_dev[dev] = p;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+        optin -= 1024;
+        if (allow_decode_smem_all(optin) != cudaSuccess) return false;
+        d.sink = static_cast<int*>(q);
+        d.sm_count = sms;
+        d.smem_limit = optin;
+        d.scratch = p;
     }
-    *scratch = g_noalloc_scratch_dev[dev];
-    *sink = g_noalloc_err_dev[dev];
+    *out = d;
     return true;
-}
-
-cudaError_t noalloc_up(int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
-    switch (nw) {
-        case 1: return launch_pdl(gemv_up_kernel<1>, grid, dim3(32), 0, s, a);
-        case 2: return launch_pdl(gemv_up_kernel<2>, grid, dim3(64), 0, s, a);
-        case 4: return launch_pdl(gemv_up_kernel<4>, grid, dim3(128), 0, s, a);
-        case 6: return launch_pdl(gemv_up_kernel<6>, grid, dim3(192), 0, s, a);
-        default: return launch_pdl(gemv_up_kernel<8>, grid, dim3(256), 0, s, a);
-    }
-}
-cudaError_t noalloc_down(int nw, dim3 grid, cudaStream_t s, const GemvArgs& a) {
-    switch (nw) {
-        case 1: return launch_pdl(gemv_down_kernel<1>, grid, dim3(32), 0, s, a);
-        case 2: return launch_pdl(gemv_down_kernel<2>, grid, dim3(64), 0, s, a);
-        case 4: return launch_pdl(gemv_down_kernel<4>, grid, dim3(128), 0, s, a);
-        case 6: return launch_pdl(gemv_down_kernel<6>, grid, dim3(192), 0, s, a);
-        default: return launch_pdl(gemv_down_kernel<8>, grid, dim3(256), 0, s, a);
-    }
 }
 
 }  // namespace
@@ -631,26 +583,17 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
     if (need > kNoallocScratchBytes) return MOE_FP4_EINVAL;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_FP4_ECUDA;
-    void* scratch = nullptr;
-    int* sink = nullptr;
-    if (!noalloc_addresses(dev, &scratch, &sink)) return MOE_FP4_ECUDA;
-    uint8_t* sp = static_cast<uint8_t*>(scratch);
-    GemvArgs a{arena, 0, 0, 0, 0, 0, 0, slot_table, layer, static_cast<int>(E), static_cast<int>(k),
+    NoallocDevice d{};
+    if (!noalloc_setup(dev, &d)) return MOE_FP4_ECUDA;
+    uint8_t* sp = static_cast<uint8_t*>(d.scratch);
+    GemvArgs a{arena, moe_fp4_slot_bytes(cfg), slot_table, layer, static_cast<int>(E), static_cast<int>(k),
                static_cast<int>(H), static_cast<int>(I), x, offsets, perm,
                reinterpret_cast<uint16_t*>(sp), reinterpret_cast<float*>(sp + h_bytes),
-               err ? reinterpret_cast<int*>(err) : sink};
-    a.slot_bytes = moe_fp4_slot_bytes(cfg);
-    a.off_w3 = I * H / 2;
-    a.off_w2 = I * H;
-    a.off_s1 = I * H + H * I / 2;
-    a.off_s3 = a.off_s1 + I * H / 32;
-    a.off_s2 = a.off_s3 + I * H / 32;
+               err ? reinterpret_cast<int*>(err) : d.sink};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const unsigned active_max = static_cast<unsigned>(ent < E ? ent : E);
-    if (noalloc_up(pick_warps(static_cast<int>(H / 128)), dim3(static_cast<unsigned>(I / 16), active_max), s, a) !=
-            cudaSuccess ||
-        noalloc_down(pick_warps(static_cast<int>(I / 128)), dim3(static_cast<unsigned>(H / 16), active_max), s, a) !=
-            cudaSuccess)
+    const int active_max = static_cast<int>(ent < E ? ent : E);
+    if (decode_forward(nullptr, a, make_slot_layout(cfg->hidden, cfg->inter), active_max, d.sm_count, d.smem_limit,
+                     s) != cudaSuccess)
         return MOE_FP4_ECUDA;
     const int n4 = T * static_cast<int>(H / 4);
     if (launch_pdl(combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s, static_cast<const float*>(a.obuf),

@@ -1,7 +1,7 @@
 // tc_prefill.cuh -- tcgen05 grouped GEMM path for large batches (prefill).
 #pragma once
 #include "common.cuh"
-#include "decode_gemv.cuh"
+#include "decode_common.cuh"
 #include "../../include/moe_fp4.h"
 
 namespace moe {

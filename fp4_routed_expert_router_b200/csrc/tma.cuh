@@ -49,14 +49,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// One bounded probe of phase `parity`: the hardware may suspend the thread
+// for up to ~0.5 ms waiting for the phase (instead of a hot spin).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
         : "memory");
     return ok != 0;
 }
@@ -67,12 +69,37 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-// Wait for phase `parity` of `bar` to complete; false after ~timeout_ns.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = 2000000000ull) {
+// Wait for phase `parity` of `bar` to complete.  Returns false at once when
+// *abort is set, and sets it (false) after ~timeout_ns: the first wait of a
+// CTA that gives up makes every later wait of that CTA return immediately, so
+// a broken pipeline costs one timeout, not one per item.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t timeout_ns = 1000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > timeout_ns) return false;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// Bounded wait until *counter > value (shared memory, written by another warp
+// of the CTA); same abort protocol as mbar_wait.
+__device__ __forceinline__ bool wait_counter_above(volatile int* counter, int value, volatile int* abort,
+                                                   uint64_t timeout_ns = 1000000000ull) {
+    if (*counter > value) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (*counter <= value) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(64);
     }
     return true;
 }
