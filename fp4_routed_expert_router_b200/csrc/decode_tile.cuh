@@ -49,7 +49,7 @@ __global__ void __launch_bounds__((RB * KS + 1) * 32, 1) gemv_tile_kernel(GemvAr
     constexpr int MATS = UP ? 2 : 1;
     constexpr int PART = MATS * 128;             // partial sums per consumer warp (16 rows x 8 tokens each)
     constexpr int TR = 16 * RB;                  // weight rows per tile
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];   // 128-byte alignment is all the row swizzle needs
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + p.stages;
     Fp4Lut* lut = reinterpret_cast<Fp4Lut*>(smem + p.off_lut);

@@ -249,6 +249,22 @@ cudaError_t decode_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& 
                     : launch_tile<false, 2, 1, 1>(c, grid, s, a, L, pd);
 }
 
+// tcgen05 path: gather x rows by expert, then the up and down GEMMs.
+cudaError_t tc_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& L, int T, cudaStream_t s) {
+    const TcPlan& p = c->tc;
+    if (!p.ready) return cudaErrorNotSupported;
+    const int rows = T * a.k;
+    cudaError_t e = launch_k(c, "gather", gather_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, s,
+                             a.x, a.perm, a.k, a.H, rows, p.xg);
+    if (e != cudaSuccess) return e;
+    const TcArgs tu = tc_args(p, a, L, T, true), td = tc_args(p, a, L, T, false);
+    if (!tu.stages || !td.stages) return cudaErrorNotSupported;
+    const dim3 grid(static_cast<unsigned>(p.sm_count)), block(kTcThreads);
+    e = launch_k(c, "tc_up", tc_gemm_kernel<true>, grid, block, tc_smem_bytes(tu), s, tu, p.map_x);
+    if (e != cudaSuccess) return e;
+    return launch_k(c, "tc_down", tc_gemm_kernel<false>, grid, block, tc_smem_bytes(td), s, td, p.map_h);
+}
+
 }  // namespace
 
 extern "C" {
@@ -299,11 +315,14 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaGetLastError();
         return bail(MOE_FP4_ENOMEM);
     }
-    if (tc_plan_create(&c->tc, *cfg) != cudaSuccess) { cudaGetLastError(); return bail(MOE_FP4_ENOMEM); }
     c->smem_optin -= 1024;   // room for the kernels' static shared memory
     if (allow_decode_smem_all(c->smem_optin) != cudaSuccess) {
         cudaGetLastError();
         return bail(MOE_FP4_ECUDA);
+    }
+    if (tc_plan_create(&c->tc, *cfg, c->d_h, c->sm_count, c->smem_optin) != cudaSuccess) {
+        cudaGetLastError();
+        return bail(MOE_FP4_ENOMEM);
     }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
@@ -449,7 +468,7 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     const int active_max = ent < E ? ent : E;
     GemvArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_h, c->d_o, c->d_err};
     const bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
-    cudaError_t e = use_tc ? tc_forward(&c->tc, a, T, s)
+    cudaError_t e = use_tc ? tc_forward(c, a, c->lay, T, s)
                            : decode_forward(c, a, c->lay, active_max, c->sm_count, c->smem_optin, s);
     if (e != cudaSuccess) return cuda_fail(c, e, "forward: expert FFN launch");
     const int n4 = T * (H / 4);

@@ -42,6 +42,18 @@ def test_tiny_layer_parity(tiny, T):
     check_y(y, y_ref)
 
 
+@pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_TC])
+@pytest.mark.parametrize("T", [1, 5, 33, 130])
+def test_tiny_forced_paths(tiny, path, T):
+    """Both expert-FFN engines on the same inputs: the register-decoded GEMV and
+    the tcgen05 grouped GEMM (token chunks of 1..128, ragged tails)."""
+    wl = tiny.wl
+    logits, mask, x, r, y = _run(tiny, T, step=1000 + T, path=path)
+    ids, w = check_routing(r, logits, wl.top_k, wl.n_experts, mask)
+    y_ref = tiny.oracle_y(0, x, ids, w, range(T))
+    check_y(y, y_ref)
+
+
 def test_tiny_zero_tokens(tiny):
     r = tiny.ctx.alloc_routing(0)
     logits = torch.empty((0, tiny.wl.n_experts), dtype=torch.float32, device="cuda")

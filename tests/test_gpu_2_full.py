@@ -50,7 +50,7 @@ def _sample_tokens(ids, n, rng):
     return sorted(pick)[: n + 3]
 
 
-@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_GEMV])
+@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_GEMV, moe.PATH_TC])
 def test_decode_b64(layer, path):
     wl = synth.WORKLOADS["decode_b64"]
     x, ids, w, y = _step(layer, wl, 64, 5, path)
@@ -58,9 +58,10 @@ def test_decode_b64(layer, path):
     check_y(y[toks], layer.oracle_y(0, x, ids, w, toks))
 
 
-def test_prefill_2048(layer):
+@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_TC])
+def test_prefill_2048(layer, path):
     wl = synth.WORKLOADS["prefill_2048"]
-    x, ids, w, y = _step(layer, wl, 2048, 7)
+    x, ids, w, y = _step(layer, wl, 2048, 7, path)
     assert len(np.unique(ids)) >= 360
     toks = _sample_tokens(ids, 8, np.random.default_rng(1))
     toks.append(2047)
