@@ -258,7 +258,7 @@ cudaError_t tc_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& L, i
                              a.x, a.perm, a.k, a.H, rows, p.xg);
     if (e != cudaSuccess) return e;
     const TcArgs tu = tc_args(p, a, L, T, true), td = tc_args(p, a, L, T, false);
-    if (!tu.stages || !td.stages) return cudaErrorNotSupported;
+    if (!tu.centries || !td.centries) return cudaErrorNotSupported;
     const dim3 grid(static_cast<unsigned>(p.sm_count)), block(kTcThreads);
     e = launch_k(c, "tc_up", tc_gemm_kernel<true>, grid, block, tc_smem_bytes(tu), s, tu, p.map_x);
     if (e != cudaSuccess) return e;

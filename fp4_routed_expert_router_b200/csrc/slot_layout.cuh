@@ -13,15 +13,19 @@
 //  down blocks  for nt in [0, H/16), f in [0, I/KBd), after all up blocks:  DB each
 //               [w2 16 rows x KBd/2][s2 16 x KBd/32]
 //
-// KBu (K extent of an up block) is the largest of 512, 256, 128 dividing H;
-// KBd is I/2 when that is a multiple of 128, else I.  Inside a block, code
-// rows whose length is a multiple of 128 bytes are swizzled: in odd rows the
-// two 64-byte halves of every 128-byte group are swapped, so that the 16-byte
-// fragment loads of rows g and g+1 (one quarter-warp phase) use disjoint
-// shared-memory banks without padding (rows of 64 mod 128 bytes alternate
-// bank halves by themselves).  Each 32-bit word of codes is also re-encoded:
-// magnitudes stay in place, the eight sign bits move (see fp4_decode.cuh).
-// Scale bytes are stored as they are.
+// KBu (KBd), the K extent of an up (down) block, is 256 when it divides H
+// (I), else 128: a block row is then 128 (64) bytes, and a 128-row tile of
+// one block is exactly four (two) 64-wide K steps of the tensor-core path.
+// Inside a block, code rows whose length is a multiple of 128 bytes are
+// swizzled: 16-byte chunk q of row r sits at q ^ ((r & 7) ^ ((r & 1) << 2)).
+// Eight consecutive rows then hold any given chunk in eight different bank
+// groups (conflict-free 16-byte loads when each lane reads one row), and rows
+// 2m, 2m+1 hold any aligned group of four chunks in opposite halves of the
+// 128 bytes (conflict-free mma fragment loads: lanes read rows g, g+1 x four
+// chunks).  Rows of 64 bytes are not swizzled (they alternate bank halves by
+// themselves).  Each 32-bit word of codes is also re-encoded: magnitudes stay
+// in place, the eight sign bits move (see fp4_decode.cuh).  Scale bytes are
+// stored as they are.
 #pragma once
 #include <cstddef>
 #include <cstdint>
@@ -41,9 +45,9 @@ __host__ __device__ inline SlotLayout make_slot_layout(int H, int I) {
     SlotLayout L;
     L.H = H;
     L.I = I;
-    L.KBu = (H % 512 == 0) ? 512 : (H % 256 == 0) ? 256 : 128;
+    L.KBu = (H % 256 == 0) ? 256 : 128;
     L.nfu = H / L.KBu;
-    L.KBd = ((I / 2) % 128 == 0) ? I / 2 : I;
+    L.KBd = (I % 256 == 0) ? 256 : 128;
     L.nfd = I / L.KBd;
     L.UB = static_cast<size_t>(32) * (L.KBu / 2 + L.KBu / 32);
     L.DB = static_cast<size_t>(16) * (L.KBd / 2 + L.KBd / 32);
@@ -54,7 +58,7 @@ __host__ __device__ inline SlotLayout make_slot_layout(int H, int I) {
 
 // Swizzled position of 16-byte chunk q of code row r (row length rowbytes).
 __host__ __device__ inline int swizzle_chunk(int q, int r, int rowbytes) {
-    return (rowbytes % 128 == 0 && (r & 1)) ? (q ^ 4) : q;
+    return (rowbytes % 128 == 0) ? (q ^ ((r & 7) ^ ((r & 1) << 2))) : q;
 }
 
 }  // namespace moe

@@ -3,30 +3,40 @@
 //
 // Per active expert e with M_e tokens (10100.com article 151357339, section
 // "moe专家的容量瓶颈"; SwiGLU reading of the unnamed activation):
-//   up    D1 = W1 X^T, D3 = W3 X^T  (128 weight rows x N tokens, K = H)
-//         h  = bf16(silu(D1) * D3)
-//   down  D  = W2 H^T               (128 weight rows x N tokens, K = I)  -> o
-// Weights are the M side (M = 128 rows per tile) and tokens the N side
-// (N <= 128, rounded up to 16), so a work item is (expert, 128-row tile,
-// chunk of <= 128 of the expert's tokens).
-//
-// One persistent CTA per SM, warp roles:
-//   warps 0-7  dequantisers: thread r (+128) decodes row r of the tile for
-//              half of a 64-wide K step straight from the slot (exact E2M1 x
-//              2^(s-127) -> bf16, fp4_decode.cuh) into the A stage, stored in
-//              the 128-byte-swizzled K-major layout the MMA reads; warps 0-3
-//              then run the epilogue from TMEM (lane r = weight row r).
-//   warp 8     TMA producer: the step's 16-row boxes of gathered token rows
-//              (x grouped by expert, or h) into the B stage, 128-byte swizzle.
-//   warp 9     MMA issuer: tcgen05.mma.cta_group::1.kind::f16 (bf16 x bf16 ->
-//              fp32 in TMEM), four K=16 instructions per matrix per step;
-//              tcgen05.commit frees the stage and, after the last step,
-//              hands the accumulators to the epilogue.
-// Stages are a ring of {A1, (A3), B} buffers with `a_full` (dequant warps),
-// `b_full` (TMA bytes) and `free` (MMA commit) mbarriers; the accumulators
-// have `acc_full` / `acc_empty`.  Every party walks the same sequence of
-// steps, so each parity wait is unambiguous; every wait is bounded and the
-// first one that gives up aborts the CTA's remaining waits.
+//   up    a1 = W1 X^T, a3 = W3 X^T, h = bf16(silu(a1) * a3)   (K = H)
+//   down  o  = W2 H^T                                         (K = I)
+// Weights are the M side of tcgen05.mma (M = 128 TMEM lanes) and tokens the
+// N side (N <= 128, rounded up to 16).  A work item is (expert, row group,
+// chunk of <= 128 of the expert's tokens):
+//   up    64 output rows: TMEM lane 32g + l holds w1 row 16g + l (l < 16) or
+//         w3 row 16g + l - 16 (l >= 16) -- exactly the two 16-row halves of
+//         slot block g -- so silu(a1) * a3 pairs lanes l and l + 16 of one
+//         warp (a shuffle, no shared memory);
+//   down  128 output rows, lane r = row r.
+// Both GEMMs therefore run the same pipeline on a 128 x 64 bf16 A tile per
+// K step.  One persistent CTA per SM, warp roles:
+//   warps 0-15   dequantisers: warp w works in TMEM lane group w % 4 and
+//                takes every fourth K step (residue w / 4); each thread
+//                decodes its row's 64 codes of the step (two 32-K chunks) from
+//                the staged FP4 blocks (exact E2M1 x 2^(s-127) -> bf16,
+//                fp4_decode.cuh) and writes them to the step's A stage in
+//                TMEM with tcgen05.st (lane = row, two bf16 per column).
+//   warps 16-19  epilogue: tcgen05.ld of the finished accumulator (double
+//                buffered), SwiGLU -> h (bf16) or o (fp32, scattered back to
+//                token-expert order), overlapping the next item's MMAs.
+//   warp 20      B producer: TMA tensor loads of the step's 16-row boxes of
+//                gathered token rows (x grouped by expert, or h), 128-byte
+//                swizzle, into shared memory.
+//   warp 21      code producer: cp.async.bulk of the item's slot blocks (all
+//                of its rows for one block's K = four steps) into a ring.
+//   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A from
+//                TMEM and B from shared memory (fp32 accumulate in TMEM), four
+//                K=16 instructions per step; tcgen05.commit frees the stage
+//                and, after the last step, hands the accumulator over.
+// Every party walks the same sequence of steps and items, so each parity wait
+// is unambiguous; every wait is bounded and the first one that gives up
+// aborts the CTA's remaining waits (MOE_FP4_ETIMEOUT), after producers have
+// let their copies in flight land.
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -40,19 +50,25 @@
 
 namespace moe {
 
-constexpr int kTcM = 128;          // weight rows per tile
-constexpr int kTcBK = 64;          // K per step (one 128-byte swizzle atom of bf16)
-constexpr int kTcNmax = 128;       // tokens per item
-constexpr int kTcDequantWarps = 8;
-constexpr int kTcThreads = (kTcDequantWarps + 2) * 32;
+constexpr int kTcM = 128;          // TMEM lanes = A rows per MMA
+constexpr int kTcBK = 64;          // K of one 128-byte swizzle atom of bf16 (four K=16 MMAs)
+constexpr int kTcSK = 128;         // K per pipeline stage (two atoms, eight MMAs)
+constexpr int kTcNmax = 128;       // tokens per item (accumulator columns)
+constexpr int kTcDequantWarps = 16;
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = (kTcDequantWarps + kTcEpiWarps + 3) * 32;   // + B producer, code producer, MMA
+constexpr int kTcStages = 4;       // A (TMEM, 64 columns each) / B (shared, 32 KB each) stages
+constexpr int kTcAccCols = 2 * kTcNmax;   // two accumulators of kTcNmax fp32 columns, then the A stages
+constexpr int kTcMaxEntries = 8;   // code ring entries at most
 
 struct TcArgs {
     GemvArgs g;
     SlotLayout L;
     int T;
-    int stages;
-    int stage_bytes;       // A (1 or 2 x 16 KB) + B (16 KB)
-    int off_stage;         // dynamic smem offset of stage 0 (1024-aligned)
+    int off_b;             // dynamic smem offset of the B ring (1024-aligned), kTcStages x 2 atoms x kTcNmax rows x 128 bytes
+    int off_code;          // offset of the code ring: centries x entry_bytes
+    int entry_bytes;       // the item's slot blocks for one block's K (4 up / 8 down blocks)
+    int centries;          // 0 when the shape does not fit
     int max_active;
 };
 
@@ -81,6 +97,16 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
+// Same, with A read from tensor memory (lane = row, two bf16 per column).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
@@ -97,6 +123,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane, then wait for the stores.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
@@ -125,19 +174,25 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* x, con
 template <bool UP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
-    constexpr int MATS = UP ? 2 : 1;
-    constexpr int A_BYTES = kTcM * 128;          // one matrix, one step: 128 rows x 64 bf16
+    constexpr int MATS = UP ? 2 : 1;             // code matrices in a slot block
+    constexpr int ROWT = UP ? 4 : 8;             // slot row tiles (16 rows) per item
+    constexpr int OUT_ROWS = UP ? 64 : 128;      // output rows per item
+    constexpr int ACOLS = kTcSK / 2;             // TMEM columns of one stage's A (bf16 pairs)
+    constexpr int BATOM = kTcNmax * 128;         // bytes of one B swizzle atom (N rows x 64 K)
+    constexpr int S = kTcStages;
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
-    // the 128-byte swizzle of the operand tiles is defined on 1024-byte atoms
-    // of the shared address space: align the working base explicitly
+    // the 128-byte swizzle of the B tiles is defined on 1024-byte atoms of the
+    // shared address space: align the working base explicitly
     uint8_t* smem = tc_smem_raw + ((1024u - (smem_u32(tc_smem_raw) & 1023u)) & 1023u);
     const GemvArgs& a = t.g;
     const SlotLayout& L = t.L;
-    uint64_t* a_full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* b_full = a_full + t.stages;
-    uint64_t* sfree = b_full + t.stages;
-    uint64_t* acc_full = sfree + t.stages;
-    uint64_t* acc_empty = acc_full + 1;
+    const int CE = t.centries;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // A decoded + B landed
+    uint64_t* sfree = full + S;
+    uint64_t* cfull = sfree + S;
+    uint64_t* cfree = cfull + CE;
+    uint64_t* acc_full = cfree + CE;             // [2]
+    uint64_t* acc_empty = acc_full + 2;          // [2]
     Fp4Lut* lut = reinterpret_cast<Fp4Lut*>(smem + 1024);              // 4 KB, 16-byte aligned
     int* act_e = reinterpret_cast<int*>(smem + 1024 + 256 * 16);
     int* act_p0 = act_e + t.max_active;
@@ -152,24 +207,33 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E;
     const int K = UP ? a.H : a.I;
-    const int rows = UP ? a.I : a.H;
-    const int n_mt = rows / kTcM;
-    const int n_steps = K / kTcBK;
+    const int n_mt = (UP ? a.I : a.H) / OUT_ROWS;
+    const int KB = UP ? L.KBu : L.KBd;           // K of one slot block = one code entry
+    const int nfb = K / KB;                      // entries per item
+    const int spe = KB / kTcSK;                  // stages per entry
+    const int n_stg = nfb * spe;                 // stages per item
+    const size_t BB = UP ? L.UB : L.DB;          // bytes of one slot block
+    const int rbb = KB / 2, sbb = KB / 32;      // code / scale bytes of a block row
 
     if (tid == 0) {
-        for (int s = 0; s < t.stages; ++s) {
-            mbar_init(&a_full[s], kTcDequantWarps);
-            mbar_init(&b_full[s], 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], kTcDequantWarps + 1);   // dequant warps + the B producer's expect_tx
             mbar_init(&sfree[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int c = 0; c < CE; ++c) {
+            mbar_init(&cfull[c], 1);
+            mbar_init(&cfree[c], kTcDequantWarps);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&acc_full[q], 1);
+            mbar_init(&acc_empty[q], kTcEpiWarps);
+        }
         abort_s = 0;
     }
-    if (warp == 0) {   // TMEM for the accumulators: 128 (or 256) columns
+    if (warp == 0) {   // all 512 TMEM columns: two accumulators, then the A stages
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&tmem_base_s)),
-                     "r"(static_cast<uint32_t>(MATS * kTcNmax)));
+                     "r"(512u));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     for (int i = tid; i < 256; i += blockDim.x) lut[i] = make_fp4_lut(static_cast<uint32_t>(i));
@@ -220,6 +284,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     }
     pdl_trigger();
     const uint32_t tmem = tmem_base_s;
+    const uint32_t tmem_a = tmem + kTcAccCols;   // A stage st at + st * ACOLS
     const int n_act = n_act_s, n_work = n_work_s, G = gridDim.x;
     const int my_items = (static_cast<int>(blockIdx.x) < n_work) ? (n_work - 1 - blockIdx.x) / G + 1 : 0;
     auto item_of = [&](int i, int& ai, int& mt, int& n0) {
@@ -235,164 +300,218 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
         mt = v / chunks;
         n0 = (v - mt * chunks) * kTcNmax;
     };
-    auto stage_a = [&](int st, int mat) { return smem + t.off_stage + static_cast<size_t>(st) * t.stage_bytes + mat * A_BYTES; };
-    auto stage_b = [&](int st) { return smem + t.off_stage + static_cast<size_t>(st) * t.stage_bytes + MATS * A_BYTES; };
+    auto code_entry = [&](int ce) { return smem + t.off_code + static_cast<size_t>(ce) * t.entry_bytes; };
+    auto stage_b = [&](int st) { return smem + t.off_b + static_cast<size_t>(st) * (2 * BATOM); };
+    const int kid = UP ? KID_TC_UP : KID_TC_DOWN;
+    const int lg = warp & 3;                                   // TMEM lane group of this warp
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * lg) << 16;
 
     if (warp < kTcDequantWarps) {
         // ------------------------------------------------------------ dequantisers
-        const int r = tid & 127, hf = tid >> 7;     // row of the tile, half of the K step
-        int gstep = 0;                              // steps walked so far (all items)
-        int items_done = 0;
+        // Warp w works in TMEM lane group w % 4 and decodes 32-K chunk w / 4 of
+        // every stage (four chunks per 128-K stage) for the 32 rows of its
+        // lanes, into the stage's A columns with one tcgen05.st.
+        const int ch = warp >> 2;                              // chunk of the stage
+        const int rr = lane & 15;                              // row inside the slot block
+        const int blk = UP ? lg : 2 * lg + (lane >> 4);        // slot block of the entry
+        const int mat = UP ? (lane >> 4) : 0;                  // w1 / w3 half of an up block
+        const int code_off = blk * static_cast<int>(BB) + mat * 16 * rbb + rr * rbb;
+        const int scale_off = blk * static_cast<int>(BB) + MATS * 16 * rbb + mat * 16 * sbb + rr * sbb;
+        int gstg = 0, gentry = 0;
         for (int i = 0; i < my_items; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int slot = act_slot[ai];
-            const int grow = mt * kTcM + r;          // weight row
-            const int rt = grow >> 4, rr = grow & 15;
-            const uint8_t* sbase = a.arena + static_cast<size_t>(slot < 0 ? 0 : slot) * a.slot_bytes;
-            if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[ai], UP ? KID_TC_UP : KID_TC_DOWN);
-            for (int s = 0; s < n_steps; ++s, ++gstep) {
-                const int st = gstep % t.stages;
-                if (gstep >= t.stages && !mbar_wait(&sfree[st], ((gstep / t.stages) - 1) & 1, abort_flag) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gstep, UP ? KID_TC_UP : KID_TC_DOWN);
-                const int k0 = s * kTcBK + hf * 32;  // first K of this thread's 32
-#pragma unroll
-                for (int mat = 0; mat < MATS; ++mat) {
+            if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[ai], kid);
+            for (int f = 0; f < nfb; ++f, ++gentry) {
+                const int ce = gentry % CE;
+                if (!mbar_wait(&cfull[ce], (gentry / CE) & 1, abort_flag) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
+                const uint8_t* ent = code_entry(ce);
+                for (int j = 0; j < spe; ++j, ++gstg) {
+                    const int st = gstg % S;
+                    if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag) && lane == 0)
+                        latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                    tc_fence_after();
+                    const int q = 4 * j + ch;                   // 32-K chunk of the block row
+                    const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off + swizzle_chunk(q, rr, rbb) * 16);
+                    const Fp4Lut lt = lut[ent[scale_off + q]];
                     uint32_t o[16];
-                    if (slot >= 0) {
-                        const uint8_t* cp;
-                        const uint8_t* sp;
-                        if (UP) {
-                            const int f = k0 / L.KBu, q = (k0 - f * L.KBu) / 32;
-                            const uint8_t* blk = sbase + (static_cast<size_t>(rt) * L.nfu + f) * L.UB;
-                            cp = blk + mat * 16 * (L.KBu / 2) + rr * (L.KBu / 2) + swizzle_chunk(q, rr, L.KBu / 2) * 16;
-                            sp = blk + 32 * (L.KBu / 2) + mat * 16 * (L.KBu / 32) + rr * (L.KBu / 32) + q;
-                        } else {
-                            const int f = k0 / L.KBd, q = (k0 - f * L.KBd) / 32;
-                            const uint8_t* blk = sbase + L.up_bytes + (static_cast<size_t>(rt) * L.nfd + f) * L.DB;
-                            cp = blk + rr * (L.KBd / 2) + swizzle_chunk(q, rr, L.KBd / 2) * 16;
-                            sp = blk + 16 * (L.KBd / 2) + rr * (L.KBd / 32) + q;
-                        }
-                        const uint4 v = ldg_stream(cp);
-                        const Fp4Lut lt = lut[__ldg(sp)];
-                        fp4_decode8(v.x, lt, o);
-                        fp4_decode8(v.y, lt, o + 4);
-                        fp4_decode8(v.z, lt, o + 8);
-                        fp4_decode8(v.w, lt, o + 12);
-                    } else {
+                    fp4_decode8(w.x, lt, o);
+                    fp4_decode8(w.y, lt, o + 4);
+                    fp4_decode8(w.z, lt, o + 8);
+                    fp4_decode8(w.w, lt, o + 12);
+                    if (slot < 0) {
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) o[q] = 0;
+                        for (int c = 0; c < 16; ++c) o[c] = 0;
                     }
-                    // row r, K chunks 4hf..4hf+3 of the 128-byte row, swizzled by r & 7
-                    uint8_t* arow = stage_a(st, mat) + r * 128;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int j = (4 * hf + c) ^ (r & 7);
-                        *reinterpret_cast<uint4*>(arow + j * 16) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-                    }
+                    tmem_st16(tmem_a + lane_addr + st * ACOLS + ch * 16, o);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[st]);
                 }
-                fence_async_smem();                    // generic stores -> tensor core reads
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[st]);
+                if (lane == 0) mbar_arrive(&cfree[ce]);
             }
-            // epilogue (warps 0-3: TMEM lanes 0-127)
-            if (warp < 4) {
-                const int p0 = act_p0[ai], m = act_m[ai];
-                const int nvalid = min(kTcNmax, m - n0);
-                if (!mbar_wait(acc_full, items_done & 1, abort_flag) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, i, UP ? KID_TC_UP : KID_TC_DOWN);
-                tc_fence_after();
-                const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-                for (int c16 = 0; c16 * 16 < nvalid; ++c16) {
-                    uint32_t v1[16], v3[16];
-                    tmem_ld16(tmem + lane_base + c16 * 16, v1);
-                    if (UP) tmem_ld16(tmem + lane_base + kTcNmax + c16 * 16, v3);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int j = c16 * 16 + q;
-                        if (j < nvalid) {
-                            const float s1 = __uint_as_float(v1[q]);
-                            if (UP) {
-                                const float s3 = __uint_as_float(v3[q]);
-                                const float hv = (slot >= 0) ? s1 / (1.0f + expf(-s1)) * s3 : 0.0f;
-                                a.hbuf[static_cast<size_t>(p0 + n0 + j) * a.I + mt * kTcM + r] = f32_to_bf16_rne(hv);
-                            } else {
-                                const int ent = __ldg(a.perm + p0 + n0 + j);
-                                a.obuf[static_cast<size_t>(ent) * a.H + mt * kTcM + r] = (slot >= 0) ? s1 : 0.0f;
-                            }
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
-            }
-            ++items_done;
         }
-    } else if (warp == kTcDequantWarps) {
-        // ------------------------------------------------------------ TMA producer (B)
-        if (lane == 0) {
-            int gstep = 0;
-            for (int i = 0; i < my_items; ++i) {
-                int ai, mt, n0;
-                item_of(i, ai, mt, n0);
-                const int nvalid = min(kTcNmax, act_m[ai] - n0);
-                const int nb = (nvalid + 15) / 16;
-                const int row0 = act_p0[ai] + n0;
-                for (int s = 0; s < n_steps; ++s, ++gstep) {
-                    const int st = gstep % t.stages;
-                    if (gstep >= t.stages && !mbar_wait(&sfree[st], ((gstep / t.stages) - 1) & 1, abort_flag))
-                        latch_error(a.err, ERR_ETIMEOUT, gstep, UP ? KID_TC_UP : KID_TC_DOWN);
-                    mbar_arrive_expect_tx(&b_full[st], static_cast<uint32_t>(nb * 16 * 128));
-                    for (int b = 0; b < nb; ++b)
-                        tma_load_2d(stage_b(st) + b * 2048, &bmap, s * kTcBK, row0 + 16 * b, &b_full[st]);
+    } else if (warp < kTcDequantWarps + kTcEpiWarps) {
+        // ------------------------------------------------------------ epilogue
+        for (int i = 0; i < my_items; ++i) {
+            int ai, mt, n0;
+            item_of(i, ai, mt, n0);
+            const int p0 = act_p0[ai], m = act_m[ai], slot = act_slot[ai];
+            const int nvalid = min(kTcNmax, m - n0);
+            const int ab = i & 1;
+            if (!mbar_wait(&acc_full[ab], (i >> 1) & 1, abort_flag) && lane == 0)
+                latch_error(a.err, ERR_ETIMEOUT, i, kid);
+            tc_fence_after();
+            for (int c16 = 0; c16 * 16 < nvalid; ++c16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + lane_addr + ab * kTcNmax + c16 * 16, v);
+                if (UP) {
+                    // lanes 0-15: a1 of rows 16 lg + lane; lanes 16-31 hold the matching a3
+#pragma unroll
+                    for (int qq = 0; qq < 16; ++qq) {
+                        const float a3 = __uint_as_float(__shfl_down_sync(0xFFFFFFFFu, v[qq], 16));
+                        const int jt = c16 * 16 + qq;
+                        if (lane < 16 && jt < nvalid) {
+                            const float a1 = __uint_as_float(v[qq]);
+                            const float hv = (slot >= 0) ? a1 / (1.0f + expf(-a1)) * a3 : 0.0f;
+                            a.hbuf[static_cast<size_t>(p0 + n0 + jt) * a.I + mt * OUT_ROWS + 16 * lg + lane] =
+                                f32_to_bf16_rne(hv);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int qq = 0; qq < 16; ++qq) {
+                        const int jt = c16 * 16 + qq;
+                        if (jt < nvalid) {
+                            const int entn = __ldg(a.perm + p0 + n0 + jt);
+                            a.obuf[static_cast<size_t>(entn) * a.H + mt * OUT_ROWS + 32 * lg + lane] =
+                                (slot >= 0) ? __uint_as_float(v[qq]) : 0.0f;
+                        }
+                    }
                 }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+    } else if (warp == kTcDequantWarps + kTcEpiWarps) {
+        // ------------------------------------------------------------ B producer
+        // The whole warp walks the loop (warp-uniform waits); lane 0 issues.
+        int gstg = 0;
+        for (int i = 0; i < my_items; ++i) {
+            int ai, mt, n0;
+            item_of(i, ai, mt, n0);
+            const int nvalid = min(kTcNmax, act_m[ai] - n0);
+            const int nb = (nvalid + 15) / 16;
+            const int row0 = act_p0[ai] + n0;
+            for (int s = 0; s < n_stg; ++s, ++gstg) {
+                const int st = gstg % S;
+                if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(2 * nb * 16 * 128));
+                    for (int at = 0; at < 2; ++at)
+                        for (int b = 0; b < nb; ++b)
+                            tma_load_2d(stage_b(st) + at * BATOM + b * 2048, &bmap, s * kTcSK + at * kTcBK,
+                                        row0 + 16 * b, &full[st]);
+                }
+                __syncwarp();
+            }
+        }
+        if (*abort_flag && lane == 0) {   // copies still in flight land before the CTA may exit
+            volatile int fresh = 0;
+            for (int st = 0; st < S && st < gstg; ++st) {
+                const int last = st + ((gstg - 1 - st) / S) * S;
+                fresh = 0;
+                mbar_wait(&full[st], (last / S) & 1, &fresh);
+            }
+        }
+    } else if (warp == kTcDequantWarps + kTcEpiWarps + 1) {
+        // ------------------------------------------------------------ code producer (FP4 blocks)
+        const uint64_t pol = policy_evict_first();
+        int gentry = 0;
+        for (int i = 0; i < my_items; ++i) {
+            int ai, mt, n0;
+            item_of(i, ai, mt, n0);
+            const int slot = act_slot[ai];
+            const uint8_t* src = a.arena + static_cast<size_t>(slot < 0 ? 0 : slot) * a.slot_bytes +
+                                 (UP ? 0 : L.up_bytes);
+            for (int f = 0; f < nfb; ++f, ++gentry) {
+                const int ce = gentry % CE;
+                if (gentry >= CE && !mbar_wait(&cfree[ce], ((gentry / CE) - 1) & 1, abort_flag) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
+                if (lane == 0) {
+                    if (slot < 0) {
+                        mbar_arrive(&cfull[ce]);
+                    } else {
+                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(ROWT * BB));
+                        for (int b = 0; b < ROWT; ++b) {   // the item's row tiles, block f
+                            const size_t rt = static_cast<size_t>(mt) * ROWT + b;
+                            bulk_g2s(code_entry(ce) + b * BB, src + (rt * nfb + f) * BB,
+                                     static_cast<uint32_t>(BB), &cfull[ce], pol);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        if (*abort_flag && lane == 0) {
+            volatile int fresh = 0;
+            for (int ce = 0; ce < CE && ce < gentry; ++ce) {
+                const int last = ce + ((gentry - 1 - ce) / CE) * CE;
+                fresh = 0;
+                mbar_wait(&cfull[ce], (last / CE) & 1, &fresh);
             }
         }
     } else {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int gstep = 0;
-            for (int i = 0; i < my_items; ++i) {
-                int ai, mt, n0;
-                item_of(i, ai, mt, n0);
-                const int nvalid = min(kTcNmax, act_m[ai] - n0);
-                const int n = (nvalid + 15) / 16 * 16;
-                const uint32_t idesc = umma_idesc_bf16(kTcM, n);
-                if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1, abort_flag))
-                    latch_error(a.err, ERR_ETIMEOUT, i, UP ? KID_TC_UP : KID_TC_DOWN);
+        int gstg = 0;
+        for (int i = 0; i < my_items; ++i) {
+            int ai, mt, n0;
+            item_of(i, ai, mt, n0);
+            const int nvalid = min(kTcNmax, act_m[ai] - n0);
+            const int n = (nvalid + 15) / 16 * 16;
+            const uint32_t idesc = umma_idesc_bf16(kTcM, n);
+            const int ab = i & 1;
+            if (i >= 2 && !mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, abort_flag) && lane == 0)
+                latch_error(a.err, ERR_ETIMEOUT, i, kid);
+            tc_fence_after();
+            const uint32_t dacc = tmem + ab * kTcNmax;
+            for (int s = 0; s < n_stg; ++s, ++gstg) {
+                const int st = gstg % S;
+                if (!mbar_wait(&full[st], (gstg / S) & 1, abort_flag) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
                 tc_fence_after();
-                for (int s = 0; s < n_steps; ++s, ++gstep) {
-                    const int st = gstep % t.stages;
-                    const uint32_t ph = (gstep / t.stages) & 1;
-                    if (!mbar_wait(&a_full[st], ph, abort_flag) || !mbar_wait(&b_full[st], ph, abort_flag))
-                        latch_error(a.err, ERR_ETIMEOUT, gstep, UP ? KID_TC_UP : KID_TC_DOWN);
-                    tc_fence_after();
-                    const uint64_t bdesc = umma_desc_sw128(smem_u32(stage_b(st)));
+                const uint64_t bdesc = umma_desc_sw128(smem_u32(stage_b(st)));
+                const uint32_t acol = tmem_a + st * ACOLS;
+                if (lane == 0) {
 #pragma unroll
-                    for (int mat = 0; mat < MATS; ++mat) {
-                        const uint64_t adesc = umma_desc_sw128(smem_u32(stage_a(st, mat)));
+                    for (int at = 0; at < 2; ++at)
 #pragma unroll
-                        for (int kk = 0; kk < kTcBK / 16; ++kk)   // +32 bytes per K=16 inside the atom
-                            umma_bf16(tmem + mat * kTcNmax, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                      (s > 0 || kk > 0) ? 1u : 0u);
-                    }
+                        for (int kk = 0; kk < kTcBK / 16; ++kk)   // K = 16: 8 TMEM columns of A, +32 bytes of B
+                            umma_bf16_ts(dacc, acol + at * (kTcBK / 2) + 8 * kk,
+                                         bdesc + static_cast<uint64_t>((at * BATOM) >> 4) + 2 * kk, idesc,
+                                         (s > 0 || at > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sfree[st]);                  // stage reusable once these MMAs are done
                 }
-                umma_commit(acc_full);                        // accumulators complete
+                __syncwarp();
             }
-            if (my_items > 0) {   // the last commits must land before TMEM is released
-                volatile int fresh = 0;
-                mbar_wait(acc_full, (my_items - 1) & 1, &fresh);
-            }
+            if (lane == 0) umma_commit(&acc_full[ab]);        // accumulator complete
+            __syncwarp();
+        }
+        if (my_items > 0 && lane == 0) {   // the last commits must land before TMEM is released
+            volatile int fresh = 0;
+            mbar_wait(&acc_full[(my_items - 1) & 1], ((my_items - 1) >> 1) & 1, &fresh);
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(static_cast<uint32_t>(MATS * kTcNmax)));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u));
 }
 
 // ------------------------------------------------------------------ host side
@@ -461,18 +580,21 @@ inline TcArgs tc_args(const TcPlan& p, const GemvArgs& g, const SlotLayout& L, i
     t.T = T;
     const int ent = T * g.k;
     t.max_active = ent < g.E ? ent : g.E;
-    const int mats = up ? 2 : 1;
-    t.stage_bytes = mats * kTcM * 128 + kTcNmax * 128;
     const int head = 1024 + 256 * 16 + 4 * (5 * t.max_active + 1 + 2 * g.E + 1);
-    t.off_stage = (head + 1023) / 1024 * 1024;
-    int stages = (p.smem_limit - 1024 - t.off_stage) / t.stage_bytes;
-    if (stages > 8) stages = 8;
-    t.stages = stages >= 2 ? stages : 0;
+    t.off_b = (head + 1023) / 1024 * 1024;
+    t.off_code = t.off_b + kTcStages * 2 * kTcNmax * 128;
+    t.entry_bytes = static_cast<int>(up ? 4 * L.UB : 8 * L.DB);
+    int ce = (p.smem_limit - 1024 - t.off_code) / t.entry_bytes;
+    if (ce > kTcMaxEntries) ce = kTcMaxEntries;
+    const int K = up ? g.H : g.I, rows = up ? g.I : g.H;
+    const int KBk = up ? L.KBu : L.KBd;
+    const bool shape_ok = (K % kTcSK == 0) && (KBk % kTcSK == 0) && (rows % (up ? 64 : kTcM) == 0);
+    t.centries = (ce >= 2 && shape_ok) ? ce : 0;
     return t;
 }
 
 inline size_t tc_smem_bytes(const TcArgs& t) {
-    return static_cast<size_t>(t.off_stage) + t.stages * t.stage_bytes + 1024;   // + alignment slack
+    return static_cast<size_t>(t.off_code) + static_cast<size_t>(t.centries) * t.entry_bytes + 1024;   // + alignment slack
 }
 
 }  // namespace moe
