@@ -3,9 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode_b1|decode_b64|prefill_2048]
 
-One step = one pass of the whole path (route + w1/w3 GEMV + SwiGLU + w2 GEMV
+One step = one pass of the whole path (route + w1/w3 GEMM + SwiGLU + w2 GEMM
 + combine) over one batch of fresh synthetic tokens of one DeepSeek-V4.1-Flash
 layer (hidden 5120, inter 2304, 384 experts resident in the arena, top-6).
+The JSON line's value is the --workload (default decode batch 1); the other
+workloads of the same layer (decode batch 64, prefill 2048 tokens) are timed
+on the same arena right after it and reported under "workloads".
 Inputs are resident in HBM when a timed step starts; L2 is flushed between
 timed steps (a 2x L2-sized write), so expert bytes really come from HBM.
 Rank 0 prints one JSON line.  Under torchrun each rank runs an independent
@@ -43,6 +46,8 @@ def parse():
     p.add_argument("--experts", type=int, default=0,
                    help="resident experts override (a smaller arena for ncu captures; 0 = the workload's)")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    p.add_argument("--only", action="store_true",
+                   help="time only --workload (skip the other workloads of the same layer)")
     return p.parse_args()
 
 
@@ -198,10 +203,209 @@ def measured_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def source_digest() -> str:
+    """Digest of the CUDA sources: a stored ncu traffic figure is used only
+    while the kernels it was taken from are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp4_routed_expert_router_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
+    recorded in profiles/traffic.json for this kernel, workload and source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(f"{kernel}@{workload}")
+    if not rec or rec.get("source_digest") != source_digest():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class Bench:
+    """One resident layer (all experts in the arena) and the timing loops."""
+
+    def __init__(self, wl, local, rank, max_tokens):
+        import torch
+        from fp4_routed_expert_router_b200 import moe
+        self.torch, self.moe = torch, moe
+        self.dev = torch.device("cuda", local)
+        self.rank = rank
+        self.wl = wl
+        self.ctx = moe.Context(wl.hidden, wl.inter, wl.n_experts, wl.top_k, 1, wl.n_experts, max_tokens,
+                               device=local)
+        staging = torch.empty(wl.expert_bytes, dtype=torch.uint8, device=self.dev)
+        for e in range(wl.n_experts):
+            moe.synth_fill_expert(staging, wl.seed, 0, e, wl.hidden, wl.inter, wl.scale_lo, wl.scale_hi)
+            self.ctx.load_expert_object(0, e, e, staging)
+        torch.cuda.synchronize()
+        rc, msg = self.ctx.last_error()
+        assert rc == moe.OK, msg
+        l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
+        self.flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=self.dev)
+        self.stream = torch.cuda.Stream(device=self.dev)
+
+    def run(self, wl, steps, warmup, graph_ok, npool, clocks=False, e2e=False):
+        torch, moe, ctx = self.torch, self.moe, self.ctx
+        T, dev, stream = wl.tokens, self.dev, self.stream
+        pool_x = torch.empty((npool, T, wl.hidden), dtype=torch.int16, device=dev)
+        pool_l = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, device=dev)
+        for i in range(npool):
+            st = self.rank * 100_000 + i
+            pool_x[i] = torch.from_numpy(synth.gen_x(wl.seed, T, wl.hidden, st).view(np.int16))
+            pool_l[i] = torch.from_numpy(synth.layer_inputs(wl, 0, st)[0])
+        x_buf = torch.empty((T, wl.hidden), dtype=torch.int16, device=dev)
+        l_buf = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
+        y_buf = torch.empty((T, wl.hidden), dtype=torch.float32, device=dev)
+        routing = ctx.alloc_routing(T)
+        flush = self.flush
+
+        def step_launch():
+            ctx.route(0, l_buf, out=routing, stream=stream)
+            ctx.forward(0, x_buf, routing, y=y_buf, stream=stream)
+
+        def stage(i):
+            x_buf.copy_(pool_x[i % npool], non_blocking=True)
+            l_buf.copy_(pool_l[i % npool], non_blocking=True)
+            flush.fill_(float(i))
+
+        out = {}
+        graph = None
+        with torch.cuda.stream(stream):
+            stage(0)
+            step_launch()
+            stream.synchronize()
+            if graph_ok:
+                try:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        step_launch()
+                    graph = g
+                except Exception as ex:  # graph capture unavailable: launch eagerly
+                    print(f"# cuda graph capture failed ({ex}); launching eagerly", file=sys.stderr)
+                    graph = None
+            run = graph.replay if graph is not None else step_launch
+            for i in range(warmup):
+                stage(i)
+                run()
+            stream.synchronize()
+            rc, msg = ctx.last_error()
+            assert rc == moe.OK, msg
+
+            # ---- timed region: K steps, events on the launching stream, L2 flushed between steps
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            if self.world > 1:
+                self.dist.barrier()
+            torch.cuda.synchronize()
+            clk = ClockSampler(dev.index) if clocks else None
+            if clk:
+                clk.__enter__()
+            for i in range(steps):
+                stage(1000 + i)
+                ev[i][0].record(stream)
+                run()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            if clk:
+                clk.__exit__(None, None, None)
+                out["clocks"] = clk.summary()
+            if self.world > 1:
+                self.dist.barrier()
+            out["total_ms"] = sum(a.elapsed_time(b) for a, b in ev)
+
+            # ---- per-kernel pass: same steps, events around every kernel
+            ctx.set_profile(True)
+            ctx.profile_read()
+            n_active = []
+            for i in range(steps):
+                stage(1000 + i)
+                step_launch()
+                n_active.append(int((routing.counts > 0).sum()))
+            recs = ctx.profile_read()
+            ctx.set_profile(False)
+            out["launches_per_step"] = len(recs) / steps
+            per_kernel = {}
+            for name, ms in recs:
+                per_kernel.setdefault(name, []).append(ms)
+            out["kernel_ms"] = {k: sum(v) / len(v) for k, v in per_kernel.items()}
+            out["active"] = float(np.mean(n_active))
+
+            if e2e:   # ---- end to end through the public API with host buffers
+                hx = torch.empty((npool, T, wl.hidden), dtype=torch.int16, pin_memory=True)
+                hl = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, pin_memory=True)
+                hx.copy_(pool_x.cpu())
+                hl.copy_(pool_l.cpu())
+                hy = torch.empty((T, wl.hidden), dtype=torch.float32, pin_memory=True)
+                e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                          for _ in range(steps)]
+                for i in range(steps):
+                    flush.fill_(float(i))
+                    e2e_ev[i][0].record(stream)
+                    x_buf.copy_(hx[i % npool], non_blocking=True)
+                    l_buf.copy_(hl[i % npool], non_blocking=True)
+                    run()
+                    hy.copy_(y_buf, non_blocking=True)
+                    e2e_ev[i][1].record(stream)
+                torch.cuda.synchronize()
+                out["e2e_ms"] = sum(a.elapsed_time(b) for a, b in e2e_ev)
+        rc, msg = ctx.last_error()
+        assert rc == moe.OK, msg
+        del graph
+        return out
+
+
+def roofline(wl, res, peaks, peak_src):
+    """Roofline of the step's dominant kernel.  Decode: the w1/w3 kernel
+    against HBM (algorithmic bytes = active experts x w1/w3 codes + scales).
+    Prefill-sized batches on the tcgen05 path: the up GEMM against the bf16
+    tensor peak (algorithmic FLOPs = 2 GEMMs x 2 H I per token-expert pair)."""
+    E, H, I, k, T = wl.n_experts, wl.hidden, wl.inter, wl.top_k, wl.tokens
+    avg, act = res["kernel_ms"], res["active"]
+    if "tc_up" in avg:
+        kern = "tc_up"
+        flops = 2.0 * 2.0 * H * I * T * k
+        achieved = flops / (avg[kern] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": stored_traffic(kern, wl.name),
+                "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed per launch)",
+                "algorithmic_flops_per_launch": flops}
+    kern = "gemv_up" if "gemv_up" in avg else max(avg, key=avg.get)
+    up_bytes_expert = 2 * (I * H // 2 + I * H // 32)
+    nbytes = act * up_bytes_expert
+    achieved = nbytes / (avg[kern] * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(kern, wl.name),
+            "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes}
+
+
+def summary(wl, res, steps, world, peaks, peak_src):
+    E, H, I, k, T = wl.n_experts, wl.hidden, wl.inter, wl.top_k, wl.tokens
+    ms = res["total_ms"] / steps
+    act = res["active"]
+    layer_bytes = act * (2 * (I * H // 2 + I * H // 32) + H * I // 2 + H * I // 32)
+    flops = 6.0 * H * I * T * k
+    return {"tok_s": T * world / (ms * 1e-3), "ms_per_step": ms,
+            "expert_bytes_per_step": layer_bytes,
+            "hbm_gbs_step": layer_bytes / (ms * 1e-3) / 1e9,
+            "hbm_frac_step": layer_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "tflops_step": flops / (ms * 1e-3) / 1e12,
+            "tensor_frac_step": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+            "active_experts_per_step": act, "kernel_ms": res["kernel_ms"],
+            "roofline": roofline(wl, res, peaks, peak_src)}
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
-    from fp4_routed_expert_router_b200 import moe
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -212,167 +416,53 @@ def run_ours(args, wl):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    # ---- arena: every expert of the layer resident, generated on the device
-    T = wl.tokens
-    ctx = moe.Context(wl.hidden, wl.inter, wl.n_experts, wl.top_k, 1, wl.n_experts, max(T, 8), device=local)
-    staging = torch.empty(wl.expert_bytes, dtype=torch.uint8, device=dev)
-    for e in range(wl.n_experts):
-        moe.synth_fill_expert(staging, wl.seed, 0, e, wl.hidden, wl.inter, wl.scale_lo, wl.scale_hi)
-        ctx.load_expert_object(0, e, e, staging)
-    torch.cuda.synchronize()
-    rc, msg = ctx.last_error()
-    assert rc == moe.OK, msg
+    # the other workloads of the same layer (same experts and seed), measured on the same arena
+    others = [] if args.only else [n for n in ("decode_b1", "decode_b64", "prefill_2048")
+                                   if n != wl.name and synth.WORKLOADS[n].n_experts == wl.n_experts]
+    max_tokens = max([wl.tokens] + [synth.WORKLOADS[n].tokens for n in others] + [8])
+    bench = Bench(wl, local, rank, max_tokens)
+    bench.world, bench.dist = world, dist
+    peaks, peak_src = measured_peaks()
 
-    # ---- a pool of fresh inputs resident in HBM (different per rank)
-    npool = 64
-    pool_x = torch.empty((npool, T, wl.hidden), dtype=torch.int16, device=dev)
-    pool_l = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, device=dev)
-    for i in range(npool):
-        st = rank * 100_000 + i
-        pool_x[i] = torch.from_numpy(synth.gen_x(wl.seed, T, wl.hidden, st).view(np.int16))
-        pool_l[i] = torch.from_numpy(synth.layer_inputs(wl, 0, st)[0])
-    x_buf = torch.empty((T, wl.hidden), dtype=torch.int16, device=dev)
-    l_buf = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
-    y_buf = torch.empty((T, wl.hidden), dtype=torch.float32, device=dev)
-    routing = ctx.alloc_routing(T)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
-    stream = torch.cuda.Stream(device=dev)
+    res = bench.run(wl, args.steps, args.warmup, not args.no_graph, 64, clocks=True, e2e=True)
+    sec = {}
+    for n in others:
+        w2 = synth.WORKLOADS[n]
+        steps2 = min(args.steps, 20)
+        r2 = bench.run(w2, steps2, max(3, min(args.warmup, 5)), not args.no_graph, 8, clocks=True)
+        sec[n] = {"steps": steps2, **summary(w2, r2, steps2, world, peaks, peak_src), "clocks": r2["clocks"]}
 
-    def step_launch():
-        ctx.route(0, l_buf, out=routing, stream=stream)
-        ctx.forward(0, x_buf, routing, y=y_buf, stream=stream)
-
-    def stage(i):
-        x_buf.copy_(pool_x[i % npool], non_blocking=True)
-        l_buf.copy_(pool_l[i % npool], non_blocking=True)
-        flush.fill_(float(i))
-
-    graph = None
-    with torch.cuda.stream(stream):
-        stage(0)
-        step_launch()
-        stream.synchronize()
-        if not args.no_graph:
-            try:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    step_launch()
-                graph = g
-            except Exception as ex:  # graph capture unavailable: launch eagerly
-                print(f"# cuda graph capture failed ({ex}); launching eagerly", file=sys.stderr)
-                graph = None
-        run = graph.replay if graph is not None else step_launch
-
-        for i in range(args.warmup):
-            stage(i)
-            run()
-        stream.synchronize()
-        rc, msg = ctx.last_error()
-        assert rc == moe.OK, msg
-
-        # ---- timed region: K steps, events on the launching stream, L2 flushed between steps
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        with ClockSampler(local) as clk:
-            for i in range(args.steps):
-                stage(1000 + i)
-                ev[i][0].record(stream)
-                run()
-                ev[i][1].record(stream)
-            torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        step_ms = [a.elapsed_time(b) for a, b in ev]
-        total_ms = sum(step_ms)
-
-        # ---- per-kernel pass: same steps, events around every kernel
-        ctx.set_profile(True)
-        ctx.profile_read()
-        n_active = []
-        for i in range(args.steps):
-            stage(1000 + i)
-            step_launch()
-            n_active.append(int((routing.counts > 0).sum()))
-        recs = ctx.profile_read()
-        ctx.set_profile(False)
-
-        # ---- end to end through the public API with host buffers
-        hx = torch.empty((npool, T, wl.hidden), dtype=torch.int16, pin_memory=True)
-        hl = torch.empty((npool, T, wl.n_experts), dtype=torch.float32, pin_memory=True)
-        hx.copy_(pool_x.cpu())
-        hl.copy_(pool_l.cpu())
-        hy = torch.empty((T, wl.hidden), dtype=torch.float32, pin_memory=True)
-        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.fill_(float(i))
-            e2e_ev[i][0].record(stream)
-            x_buf.copy_(hx[i % npool], non_blocking=True)
-            l_buf.copy_(hl[i % npool], non_blocking=True)
-            run()
-            hy.copy_(y_buf, non_blocking=True)
-            e2e_ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    rc, msg = ctx.last_error()
-    assert rc == moe.OK, msg
-
+    total_ms, e2e_ms = res["total_ms"], res["e2e_ms"]
     if world > 1:
         t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms, e2e_ms = float(t[0]), float(t[1])
+        res["total_ms"] = total_ms
 
-    # ---- roofline of the dominant kernel (w1/w3 stream)
-    per_kernel = {}
-    for name, ms in recs:
-        per_kernel.setdefault(name, []).append(ms)
-    avg = {k: sum(v) / len(v) for k, v in per_kernel.items()}
-    peaks, peak_src = measured_peaks()
-    E, H, I, k = wl.n_experts, wl.hidden, wl.inter, wl.top_k
-    up_bytes_expert = 2 * (I * H // 2 + I * H // 32)
-    down_bytes_expert = H * I // 2 + H * I // 32
-    act = float(np.mean(n_active))   # active experts per step, from the routing counts
-    dominant = "gemv_up" if "gemv_up" in avg else max(avg, key=avg.get)
-    dom_bytes = act * (up_bytes_expert if dominant == "gemv_up" else down_bytes_expert)
-    achieved = dom_bytes / (avg[dominant] * 1e-3) / 1e9
-    layer_bytes = act * (up_bytes_expert + down_bytes_expert)
-    fwd_ms = sum(avg.get(n, 0.0) for n in ("gemv_up", "gemv_down", "combine"))
-
-    ms_per_step = total_ms / args.steps
+    s = summary(wl, res, args.steps, world, peaks, peak_src)
+    T = wl.tokens
     toks = T * args.steps * world
-    value = toks / (total_ms * 1e-3)
     line = {
-        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(wl, graph is not None),
-        "hbm_gbs_step": layer_bytes / (ms_per_step * 1e-3) / 1e9,
-        "hbm_frac_step": layer_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "kernel_ms": avg,
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "peak_source": f"{peak_src} hbm_gbs",
-                     "algorithmic_bytes_per_launch": dom_bytes},
-        "layer_roofline": {"bytes_per_step": layer_bytes, "forward_kernels_ms": fwd_ms,
-                           "achieved_gbs": layer_bytes / (fwd_ms * 1e-3) / 1e9 if fwd_ms else None,
-                           "frac": (layer_bytes / (fwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if fwd_ms else None},
-        "active_experts_per_step": act,
+        "metric": METRIC, "value": toks / (total_ms * 1e-3), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, not args.no_graph),
+        "hbm_gbs_step": s["hbm_gbs_step"], "hbm_frac_step": s["hbm_frac_step"],
+        "kernel_ms": s["kernel_ms"],
+        "roofline": s["roofline"],
+        "active_experts_per_step": s["active_experts_per_step"],
         "e2e": {"value": toks / (e2e_ms * 1e-3), "unit": "tok/s",
                 "h2d_bytes_per_step": T * (wl.hidden * 2 + wl.n_experts * 4),
                 "d2h_bytes_per_step": T * wl.hidden * 4},
-        "gpu_launches": 4 * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": int(round(res["launches_per_step"] * args.steps)),
+        "clocks": res["clocks"],
+        "workloads": sec,
     }
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
-    ctx.close()
+    bench.ctx.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
