@@ -203,28 +203,34 @@ def measured_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def source_digest() -> str:
-    """Digest of the CUDA sources: a stored ncu traffic figure is used only
-    while the kernels it was taken from are unchanged."""
+def source_digest(files) -> str:
+    """Digest of the listed CUDA sources (sha256 over name, NUL, bytes, in list
+    order): a stored ncu traffic figure is used only while the sources of the
+    kernel it was taken from are unchanged."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp4_routed_expert_router_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in files:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def stored_traffic(kernel: str, workload: str):
     """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
-    recorded in profiles/traffic.json for this kernel, workload and source."""
+    recorded in profiles/traffic.json for this kernel and workload, or None
+    when there is none or its sources changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f).get(f"{kernel}@{workload}")
-    if not rec or rec.get("source_digest") != source_digest():
+    if not rec:
+        return None
+    try:
+        if source_digest(rec["files"]) != rec["source_digest"]:
+            return None
+    except OSError:
         return None
     return rec.get("bytes_per_launch")
 
@@ -363,28 +369,32 @@ class Bench:
 
 
 def roofline(wl, res, peaks, peak_src):
-    """Roofline of the step's dominant kernel.  Decode: the w1/w3 kernel
-    against HBM (algorithmic bytes = active experts x w1/w3 codes + scales).
-    Prefill-sized batches on the tcgen05 path: the up GEMM against the bf16
-    tensor peak (algorithmic FLOPs = 2 GEMMs x 2 H I per token-expert pair)."""
+    """Roofline of the step's dominant kernel, the w1/w3 one (gemv_up or
+    tc_up).  Algorithmic bytes = active experts x w1/w3 codes + scales;
+    algorithmic FLOPs = 2 GEMMs x 2 H I per token-expert pair.  The bound is
+    the one the arithmetic intensity selects against the measured ridge
+    point; the tensor-core path also reports its fraction of the bf16 peak."""
     E, H, I, k, T = wl.n_experts, wl.hidden, wl.inter, wl.top_k, wl.tokens
     avg, act = res["kernel_ms"], res["active"]
-    if "tc_up" in avg:
-        kern = "tc_up"
-        flops = 2.0 * 2.0 * H * I * T * k
-        achieved = flops / (avg[kern] * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        return {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": stored_traffic(kern, wl.name),
-                "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed per launch)",
-                "algorithmic_flops_per_launch": flops}
-    kern = "gemv_up" if "gemv_up" in avg else max(avg, key=avg.get)
-    up_bytes_expert = 2 * (I * H // 2 + I * H // 32)
-    nbytes = act * up_bytes_expert
-    achieved = nbytes / (avg[kern] * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(kern, wl.name),
-            "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes}
+    kern = "tc_up" if "tc_up" in avg else ("gemv_up" if "gemv_up" in avg else max(avg, key=avg.get))
+    sec = avg[kern] * 1e-3
+    nbytes = act * 2 * (I * H // 2 + I * H // 32)
+    flops = 2.0 * 2.0 * H * I * T * k
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    gbs, tfs = nbytes / sec / 1e9, flops / sec / 1e12
+    out_hbm = {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+               "frac": gbs / peaks["hbm_gbs"], "traffic": stored_traffic(kern, wl.name),
+               "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
+               "intensity_flop_per_byte": flops / nbytes, "ridge_flop_per_byte": ridge}
+    out_tc = {"bound": "tensor", "kernel": kern, "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+              "frac": tfs / peaks["bf16_tflops"], "traffic": stored_traffic(kern, wl.name),
+              "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed per launch)",
+              "algorithmic_flops_per_launch": flops}
+    hbm_bound = flops / nbytes < ridge
+    main = dict(out_hbm if hbm_bound else out_tc)
+    if kern == "tc_up":
+        main["other"] = out_tc if hbm_bound else out_hbm
+    return main
 
 
 def summary(wl, res, steps, world, peaks, peak_src):
