@@ -413,6 +413,16 @@ def summary(wl, res, steps, world, peaks, peak_src):
             "roofline": roofline(wl, res, peaks, peak_src)}
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of per-rank timings over the process group (every
+    rank takes this same collective step).  The multi-GPU number is the
+    slowest rank's device time."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -444,9 +454,7 @@ def run_ours(args, wl):
 
     total_ms, e2e_ms = res["total_ms"], res["e2e_ms"]
     if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
         res["total_ms"] = total_ms
 
     s = summary(wl, res, args.steps, world, peaks, peak_src)
