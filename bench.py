@@ -8,7 +8,8 @@ One step = one pass of the whole path (route + w1/w3 GEMM + SwiGLU + w2 GEMM
 layer (hidden 5120, inter 2304, 384 experts resident in the arena, top-6).
 The JSON line's value is the --workload (default decode batch 1); the other
 workloads of the same layer (decode batch 64, prefill 2048 tokens) are timed
-on the same arena right after it and reported under "workloads".
+on the same arena right after it, then the 40-layer stack (batch 1 and 8, its
+own 115.8 GB arena), all reported under "workloads".
 Inputs are resident in HBM when a timed step starts; L2 is flushed between
 timed steps (a 2x L2-sized write), so expert bytes really come from HBM.
 Rank 0 prints one JSON line.  Under torchrun each rank runs an independent
@@ -368,6 +369,118 @@ class Bench:
         return out
 
 
+def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
+    """The 40-layer expert-FFN stack: each layer keeps its n_keep most popular
+    experts in one arena (40 x 154 = 6,160 slots, 115.8 GB), the router is
+    masked to the kept set, and x <- bf16(x + y) between layers, in place.
+    One step = 40 x (route + forward) for one batch of fresh tokens, captured
+    in one CUDA graph.  Returns {workload name: summary} for each of ``wls``
+    (same layers and experts, different batch sizes), sharing one arena."""
+    import torch
+    from fp4_routed_expert_router_b200 import moe
+    wl0 = wls[0]
+    dev = torch.device("cuda", local)
+    L, E, H, I, k = wl0.n_layers, wl0.n_experts, wl0.hidden, wl0.inter, wl0.top_k
+    kept = wl0.n_keep
+    tmax = max(w.tokens for w in wls)
+    ctx = moe.Context(H, I, E, k, L, kept * L, max(tmax, 8), device=local)
+    staging = torch.empty(wl0.expert_bytes, dtype=torch.uint8, device=dev)
+    slot = 0
+    for layer in range(L):
+        for e in synth.resident_experts(wl0, layer):
+            moe.synth_fill_expert(staging, wl0.seed, layer, int(e), H, I, wl0.scale_lo, wl0.scale_hi)
+            ctx.load_expert_object(layer, int(e), slot, staging)
+            slot += 1
+    del staging
+    masks = [torch.from_numpy(synth.keep_mask(wl0.seed, l, E, kept)).to(dev) for l in range(L)]
+    torch.cuda.synchronize()
+    rc, msg = ctx.last_error()
+    assert rc == moe.OK, msg
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+    for wl in wls:
+        T = wl.tokens
+        npool = 8
+        pool_x = torch.empty((npool, T, H), dtype=torch.int16, device=dev)
+        pool_l = torch.empty((npool, L, T, E), dtype=torch.float32, device=dev)
+        for i in range(npool):
+            st = rank * 100_000 + i
+            pool_x[i] = torch.from_numpy(synth.gen_x(wl.seed, T, H, st).view(np.int16))
+            for l in range(L):
+                pool_l[i, l] = torch.from_numpy(synth.layer_inputs(wl, l, st)[0])
+        x_buf = torch.empty((T, H), dtype=torch.int16, device=dev)
+        l_buf = torch.empty((L, T, E), dtype=torch.float32, device=dev)
+        y_buf = torch.empty((T, H), dtype=torch.float32, device=dev)
+        routes = [ctx.alloc_routing(T) for _ in range(L)]
+
+        def step_launch():
+            for l in range(L):
+                ctx.route(l, l_buf[l], masks[l], out=routes[l], stream=stream)
+                ctx.forward(l, x_buf, routes[l], y=y_buf, x_out=x_buf, stream=stream)
+
+        def stage(i):
+            x_buf.copy_(pool_x[i % npool], non_blocking=True)
+            l_buf.copy_(pool_l[i % npool], non_blocking=True)
+            flush.fill_(float(i))
+
+        graph = None
+        with torch.cuda.stream(stream):
+            stage(0)
+            step_launch()
+            stream.synchronize()
+            if graph_ok:
+                try:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        step_launch()
+                    graph = g
+                except Exception as ex:
+                    print(f"# cuda graph capture failed ({ex}); launching eagerly", file=sys.stderr)
+            run = graph.replay if graph is not None else step_launch
+            for i in range(warmup):
+                stage(i)
+                run()
+            stream.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            clk = ClockSampler(dev.index)
+            clk.__enter__()
+            active = []
+            for i in range(steps):
+                stage(1000 + i)
+                ev[i][0].record(stream)
+                run()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            clk.__exit__(None, None, None)
+            if world > 1:
+                dist.barrier()
+            for r in routes:     # active experts of the last step, per layer
+                active.append(int((r.counts > 0).sum()))
+        rc, msg = ctx.last_error()
+        assert rc == moe.OK, msg
+        total_ms = sum(a.elapsed_time(b) for a, b in ev)
+        if world > 1:
+            total_ms = max_over_ranks([total_ms], dist, dev)[0]
+        ms = total_ms / steps
+        nbytes = sum(active) * wl.expert_bytes
+        out[wl.name] = {"steps": steps, "tok_s": T * world / (ms * 1e-3), "ms_per_step": ms,
+                        "layers": L, "slots": kept * L, "arena_bytes": kept * L * wl.expert_bytes,
+                        "expert_bytes_per_step": nbytes, "active_experts_per_step": sum(active),
+                        "hbm_gbs_step": nbytes / (ms * 1e-3) / 1e9,
+                        "hbm_frac_step": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "launch": "one cuda graph of 40 x (route + forward)" if graph is not None else "eager",
+                        "clocks": clk.summary()}
+        del graph
+    ctx.close()
+    return out
+
+
 def roofline(wl, res, peaks, peak_src):
     """Roofline of the step's dominant kernel, the w1/w3 one (gemv_up or
     tc_up).  Algorithmic bytes = active experts x w1/w3 codes + scales;
@@ -452,6 +565,14 @@ def run_ours(args, wl):
         r2 = bench.run(w2, steps2, max(3, min(args.warmup, 5)), not args.no_graph, 8, clocks=True)
         sec[n] = {"steps": steps2, **summary(w2, r2, steps2, world, peaks, peak_src), "clocks": r2["clocks"]}
 
+    if not args.only and wl.n_experts == synth.WORKLOADS["stack40_b1"].n_experts:
+        bench.ctx.close()
+        bench.ctx = None
+        torch.cuda.empty_cache()
+        stack = [synth.WORKLOADS[n] for n in ("stack40_b1", "stack40_b8")]
+        sec.update(run_stack(stack, local, rank, min(args.steps, 20), max(3, min(args.warmup, 5)),
+                             not args.no_graph, peaks, world, dist))
+
     total_ms, e2e_ms = res["total_ms"], res["e2e_ms"]
     if world > 1:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
@@ -480,7 +601,8 @@ def run_ours(args, wl):
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    bench.ctx.close()
+    if bench.ctx is not None:
+        bench.ctx.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

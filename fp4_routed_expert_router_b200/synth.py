@@ -229,6 +229,10 @@ WORKLOADS = {
                            notes="one V4.1-Flash layer, 384 experts resident, batch 64"),
     "prefill_2048": Workload("prefill_2048", 5120, 2304, 384, 6, 2048, zipf_alpha=0.47,
                              notes="one V4.1-Flash layer, 2048-token prefill chunk"),
+    "drafter_b1": Workload("drafter_b1", 5120, 2304, 128, 3, 1, zipf_alpha=0.5,
+                           notes="drafter-shaped MoE (128 experts, top-3) at the layer's hidden/inter, batch 1"),
+    "drafter_b256": Workload("drafter_b256", 5120, 2304, 128, 3, 256, zipf_alpha=0.5,
+                             notes="drafter-shaped MoE (128 experts, top-3), batch 256"),
     "stack40_b1": Workload("stack40_b1", 5120, 2304, 384, 6, 1, n_layers=40, zipf_alpha=0.5,
                            n_keep=154, notes="40 layers x 154 kept experts, batch 1"),
     "stack40_b8": Workload("stack40_b8", 5120, 2304, 384, 6, 8, n_layers=40, zipf_alpha=0.5,
