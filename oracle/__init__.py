@@ -54,6 +54,10 @@ def lib():
         _lib.oracle_moe_forward.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_int, P, P, P,
                                             ctypes.c_int, P]
+        _lib.oracle_moe_saliency.restype = ctypes.c_int
+        _lib.oracle_moe_saliency.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, P, P, P,
+                                            ctypes.c_int, P]
         _lib.oracle_residual.restype = None
         _lib.oracle_residual.argtypes = [P, P, ctypes.c_size_t]
         _lib.oracle_max_threads.restype = ctypes.c_int
@@ -149,6 +153,26 @@ def moe_forward(x: np.ndarray, ids: np.ndarray, w: np.ndarray, objs: dict, n_exp
     if rc != 0:
         raise ValueError(f"oracle_moe_forward failed ({rc})")
     return y
+
+
+def saliency(x: np.ndarray, ids: np.ndarray, w: np.ndarray, objs: dict, n_experts: int, hidden: int, inter: int,
+             n_threads: int = 0) -> np.ndarray:
+    """Per-expert saliency float64 [E]: sum of w[t,j] * ||o_{t,j}||_2 over the
+    entries routed to each expert (zero for experts nobody chose)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, k = ids.shape
+    keep = [np.ascontiguousarray(objs[e], dtype=np.uint8) if e in objs else None
+            for e in range(n_experts)]
+    ptrs = (ctypes.c_void_p * n_experts)(*[(v.ctypes.data if v is not None else None)
+                                           for v in keep])
+    sal = np.zeros(n_experts, dtype=np.float64)
+    rc = lib().oracle_moe_saliency(_p(x), T, hidden, inter, n_experts, k, _p(ids), _p(w),
+                                   ctypes.cast(ptrs, ctypes.c_void_p), n_threads, _p(sal))
+    if rc != 0:
+        raise ValueError(f"oracle_moe_saliency failed ({rc})")
+    return sal
 
 
 def residual(x: np.ndarray, y: np.ndarray) -> np.ndarray:

@@ -34,6 +34,11 @@
  *    article's saliency, router weight x expert output, section
  *    "选哪些专家：频率 vs Saliency", implies the router-weighted sum).
  *  - Residual between stacked layers: x <- bf16_rne(x + y).
+ *  - Expert saliency (10100.com article 151357339, section
+ *    "选哪些专家：频率 vs Saliency": router weight times the L2 norm of the
+ *    expert's output, summed over the tokens of a corpus):
+ *    S[e] += sum over (t, j) with ids[t,j] = e of w[t,j] * ||o_{t,j}||_2,
+ *    o_{t,j} the expert's output row for token t as in the FFN above.
  */
 #include <math.h>
 #include <stdint.h>
@@ -275,6 +280,44 @@ int oracle_moe_forward(const uint16_t *x, int T, int H, int I, int E, int k,
                 acc += w[(size_t)t * k + j] * o[((size_t)t * k + j) * H + n];
             y[(size_t)t * H + n] = acc;
         }
+    free(o);
+    return 0;
+}
+
+/* Saliency accumulation: sal[e] += sum over entries p = t*k + j routed to e of
+ * w[p] * ||o_p||_2, o_p = expert ids[p]'s output for token t (fp64 throughout).
+ * Same expert layout and error codes as oracle_moe_forward. */
+int oracle_moe_saliency(const uint16_t *x, int T, int H, int I, int E, int k,
+                        const int32_t *ids, const double *w,
+                        const uint8_t *const *objs, int n_threads, double *sal)
+{
+    size_t w13 = (size_t)I * (H / 2), w2b = (size_t)H * (I / 2);
+    size_t s13 = (size_t)I * (H / 32);
+    for (int i = 0; i < T * k; ++i)
+        if (ids[i] < 0 || ids[i] >= E || !objs[ids[i]]) return -1;
+    double *norm = (double *)malloc(sizeof(double) * (size_t)(T * k > 0 ? T * k : 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)(T * k > 0 ? T * k : 1) * H);
+    if (!norm || !o) {
+        free(norm);
+        free(o);
+        return -2;
+    }
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int p = 0; p < T * k; ++p) {
+        const uint8_t *b = objs[ids[p]];
+        expert_ptrs ep = {b, b + 2 * w13 + w2b, b + w13, b + 2 * w13 + w2b + s13,
+                          b + 2 * w13, b + 2 * w13 + w2b + 2 * s13};
+        double *op = o + (size_t)p * H;
+        expert_ffn(x + (size_t)(p / k) * H, H, I, &ep, NULL, op);
+        double ss = 0.0;
+        for (int n = 0; n < H; ++n) ss += op[n] * op[n];
+        norm[p] = sqrt(ss);
+    }
+    for (int p = 0; p < T * k; ++p) sal[ids[p]] += w[p] * norm[p];
+    free(norm);
     free(o);
     return 0;
 }

@@ -287,3 +287,54 @@ def test_residual_rounds_once():
     ref = [helpers.bf16_exact_round(float(a + b))
            for a, b in zip(helpers.bf16_bits_to_f64(x).ravel(), y.ravel())]
     np.testing.assert_array_equal(helpers.bf16_bits_to_f64(out).ravel(), ref)
+
+
+def test_saliency_brute_force_dense():
+    # saliency = sum over entries routed to e of w * ||o||_2, with o from dense
+    # table-decoded matrices (independent of the oracle's decoder)
+    H, I, E, k, T = 64, 96, 8, 3, 7
+    objs = _tiny_layer(60, H, I, E)
+    lay = synth.expert_layout(H, I)
+    x = synth.gen_x(61, T, H)
+    logits = np.random.default_rng(62).standard_normal((T, E)).astype(np.float32)
+    ids, w = oracle.route(logits, k)
+    sal = oracle.saliency(x, ids, w, objs, E, H, I)
+
+    def part(obj, name):
+        off, (r, c) = lay[name]
+        return obj[off:off + r * c].reshape(r, c)
+
+    ref = np.zeros(E)
+    for t in range(T):
+        xd = helpers.bf16_bits_to_f64(x[t])
+        for j in range(k):
+            e = int(ids[t, j])
+            ob = objs[e]
+            W1 = helpers.dense_from_table(part(ob, "w1"), part(ob, "s1"))
+            W3 = helpers.dense_from_table(part(ob, "w3"), part(ob, "s3"))
+            W2 = helpers.dense_from_table(part(ob, "w2"), part(ob, "s2"))
+            h = np.array([helpers.bf16_exact_round(float(v)) for v in _silu(W1 @ xd) * (W3 @ xd)])
+            ref[e] += w[t, j] * math.sqrt(float(np.sum((W2 @ h) ** 2)))
+    np.testing.assert_allclose(sal, ref, rtol=1e-11, atol=0)
+    unused = np.setdiff1d(np.arange(E), np.unique(ids))
+    assert np.all(sal[unused] == 0.0)
+
+
+def test_saliency_power_of_two_invariants():
+    # w2 scales + 1 => every output doubles => saliency doubles exactly;
+    # doubling the router weights doubles it too
+    H, I, E, k, T = 64, 96, 6, 2, 5
+    objs = _tiny_layer(70, H, I, E)
+    lay = synth.expert_layout(H, I)
+    x = synth.gen_x(71, T, H)
+    logits = np.random.default_rng(72).standard_normal((T, E)).astype(np.float32)
+    ids, w = oracle.route(logits, k)
+    sal = oracle.saliency(x, ids, w, objs, E, H, I)
+    off, (r, c) = lay["s2"]
+    bumped = {}
+    for e, ob in objs.items():
+        b = ob.copy()
+        b[off:off + r * c] += 1
+        bumped[e] = b
+    np.testing.assert_array_equal(oracle.saliency(x, ids, w, bumped, E, H, I), 2.0 * sal)
+    np.testing.assert_array_equal(oracle.saliency(x, ids, 2.0 * w, objs, E, H, I), 2.0 * sal)
