@@ -86,4 +86,42 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* obuf, const f
     }
 }
 
+// ||o_p||_2 of each per-entry output row: one warp per row, lanes sum
+// strided squares in index order, then a fixed xor tree (deterministic).
+__global__ void __launch_bounds__(256) entry_norm_kernel(const float* obuf, int n_ent, int H, float* norms) {
+    pdl_wait();
+    pdl_trigger();
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (row >= n_ent) return;
+    const float4* r = reinterpret_cast<const float4*>(obuf + static_cast<size_t>(row) * H);
+    float s = 0.f;
+    for (int i = lane; i < H / 4; i += 32) {
+        const float4 v = __ldcg(r + i);
+        s = fmaf(v.x, v.x, s);
+        s = fmaf(v.y, v.y, s);
+        s = fmaf(v.z, v.z, s);
+        s = fmaf(v.w, v.w, s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    if (lane == 0) norms[row] = sqrtf(s);
+}
+
+// saliency[e] += sum over e's grouped entries of w * norm, in perm order, fp64.
+__global__ void __launch_bounds__(128) saliency_kernel(const float* norms, const float* w, const int32_t* offsets,
+                                                       const int32_t* perm, int E, double* sal) {
+    pdl_wait();
+    pdl_trigger();
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const int p0 = __ldg(offsets + e), p1 = __ldg(offsets + e + 1);
+    if (p1 <= p0) return;
+    double acc = 0.0;
+    for (int p = p0; p < p1; ++p) {
+        const int ent = __ldg(perm + p);
+        acc += static_cast<double>(__ldg(w + ent)) * static_cast<double>(norms[ent]);
+    }
+    sal[e] += acc;
+}
+
 }  // namespace moe

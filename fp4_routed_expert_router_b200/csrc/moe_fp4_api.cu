@@ -35,6 +35,7 @@ struct moe_fp4_ctx {
     uint8_t* d_staging = nullptr;      // one expert, checkpoint layout
     uint16_t* d_h = nullptr;           // [max_tokens*k, I] bf16
     float* d_o = nullptr;              // [max_tokens*k, H] fp32
+    float* d_norm = nullptr;           // [max_tokens*k] fp32 (saliency)
     int* d_err = nullptr;              // error word [4]
     unsigned int* d_ticket = nullptr;  // route kernel ticket
     std::vector<int32_t> h_table;      // host mirror of d_table
@@ -310,6 +311,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaMalloc(&c->d_staging, c->slot_bytes) != cudaSuccess ||
         cudaMalloc(&c->d_h, sizeof(uint16_t) * ent * I) != cudaSuccess ||
         cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
+        cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
         cudaGetLastError();
@@ -344,6 +346,7 @@ void moe_fp4_destroy(moe_fp4_ctx* c) {
     cudaFree(c->d_staging);
     cudaFree(c->d_h);
     cudaFree(c->d_o);
+    cudaFree(c->d_norm);
     cudaFree(c->d_err);
     cudaFree(c->d_ticket);
     tc_plan_destroy(&c->tc);
@@ -475,6 +478,25 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
                  static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
     if (e != cudaSuccess) return cuda_fail(c, e, "forward: combine launch");
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_saliency(moe_fp4_ctx* c, int T, const float* weights, const int32_t* offsets,
+                                const int32_t* perm, double* saliency, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (T < 0 || T > g.max_tokens) return host_fail(c, MOE_FP4_EINVAL, "saliency: T %d out of range", T);
+    if (T == 0) return MOE_FP4_OK;
+    if (!weights || !offsets || !perm || !saliency) return host_fail(c, MOE_FP4_EINVAL, "saliency: NULL argument");
+    cudaSetDevice(c->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int n_ent = T * g.top_k;
+    cudaError_t e = launch_k(c, "entry_norm", entry_norm_kernel, dim3((n_ent * 32 + 255) / 256), dim3(256), 0, s,
+                             static_cast<const float*>(c->d_o), n_ent, g.hidden, c->d_norm);
+    if (e != cudaSuccess) return cuda_fail(c, e, "saliency: norm launch");
+    e = launch_k(c, "saliency", saliency_kernel, dim3((g.n_experts + 127) / 128), dim3(128), 0, s,
+                 static_cast<const float*>(c->d_norm), weights, offsets, perm, g.n_experts, saliency);
+    if (e != cudaSuccess) return cuda_fail(c, e, "saliency: launch");
     return MOE_FP4_OK;
 }
 

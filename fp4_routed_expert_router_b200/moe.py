@@ -24,7 +24,7 @@ OPT_PATH, OPT_PROFILE = 1, 2
 # every symbol include/moe_fp4.h declares
 EXPORTS = ("moe_fp4_slot_bytes", "moe_fp4_create", "moe_fp4_destroy", "moe_fp4_arena",
            "moe_fp4_set_option", "moe_fp4_profile_read", "moe_fp4_load_expert_slot", "moe_fp4_route",
-           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc")
+           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency")
 
 
 class MoeError(RuntimeError):
@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH):
         L.moe_fp4_route.argtypes = [P, I32, P, P, I32, P, P, P, P, P, P]
         L.moe_fp4_forward.restype = I32
         L.moe_fp4_forward.argtypes = [P, I32, P, I32, P, P, P, P, P, P, P, P]
+        L.moe_fp4_saliency.restype = I32
+        L.moe_fp4_saliency.argtypes = [P, I32, P, P, P, P, P]
         L.moe_fp4_last_error.restype = I32
         L.moe_fp4_last_error.argtypes = [P, ctypes.c_char_p, SZ]
         L.moe_fp4_forward_noalloc.restype = I32
@@ -234,6 +236,17 @@ class Context:
                                       _ptr(r.offsets), _ptr(r.perm), _ptr(y), _ptr(x_out), _stream(stream))
         self._check(rc, "forward")
         return y
+
+
+    def saliency(self, r: Routing, sal: torch.Tensor, stream=None) -> torch.Tensor:
+        """Accumulate per-expert saliency (fp64 [E] device tensor) of the last
+        forward on this context: sal[e] += sum of weight * ||expert output||_2
+        over the entries routed to e.  Call after forward, same stream."""
+        T = r.ids.shape[0]
+        rc = self.lib.moe_fp4_saliency(self.h, T, _ptr(r.weights), _ptr(r.offsets), _ptr(r.perm), _ptr(sal),
+                                       _stream(stream))
+        self._check(rc, "saliency")
+        return sal
 
 
 def _data_ptr(t) -> int:

@@ -185,6 +185,28 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, i
                                const int32_t *perm, float *y, uint16_t *x_out, void *stream);
 
 /*
+ * Expert saliency of the last forward (10100.com article 151357339, section
+ * "选哪些专家：频率 vs Saliency": router weight times the L2 norm of the
+ * expert's output, summed over a corpus, used to rank experts for pruning):
+ *   saliency[e] += sum over the entries p = t*k + j routed to e of
+ *                  weights[p] * ||o_p||_2
+ * where o_p is expert ids[p]'s fp32 output row for token t, as the last
+ * moe_fp4_forward on this context left it in the workspace.  Call it on the
+ * same stream after that forward (same T, weights, offsets, perm) and before
+ * the next forward on the context.  Norms are fp32 sums in a fixed order;
+ * each expert's entries are added in grouped (perm) order in fp64, and each
+ * expert's total is added once to saliency[e], so the result does not depend
+ * on the schedule.  Experts without entries are left unchanged.
+ *  weights   fp32 [T, k], offsets int32 [E+1], perm int32 [T*k]: device.
+ *  saliency  fp64 [E] device accumulator, owned by the caller (zero it to
+ *            start a corpus).
+ * T = 0 does nothing.  Errors: EINVAL (bad T or NULL pointer), ECUDA.
+ */
+moe_fp4_status moe_fp4_saliency(moe_fp4_ctx *ctx, int T, const float *weights,
+                                const int32_t *offsets, const int32_t *perm,
+                                double *saliency, void *stream);
+
+/*
  * Synchronise the device, read and clear the device error word.  Returns the
  * first latched status (OK if none) and writes a one-line description into
  * msg (n bytes, may be NULL).  Host-side errors of the last failing call are

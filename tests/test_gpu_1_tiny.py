@@ -131,3 +131,26 @@ def test_residual_output(tiny):
     diff = np.abs(got - x_ref.astype(np.int32))      # same sign: bit distance = ulps
     assert diff.max() <= 1
     assert (diff == 0).mean() > 0.97
+
+
+@pytest.mark.parametrize("path,T", [(moe.PATH_GEMV, 17), (moe.PATH_TC, 130), (moe.PATH_AUTO, 200)])
+def test_tiny_saliency(tiny, path, T):
+    """Per-expert saliency (router weight x ||expert output||_2, summed) of a
+    forward against the oracle; experts nobody chose stay untouched; a second
+    call on the same forward adds the same amount again (exactly, in fp64)."""
+    wl = tiny.wl
+    logits, mask, x, r, y = _run(tiny, T, step=2000 + T, path=path)
+    ids, w = check_routing(r, logits, wl.top_k, wl.n_experts, mask)
+    sal = torch.zeros(wl.n_experts, dtype=torch.float64, device="cuda")
+    tiny.ctx.saliency(r, sal)
+    s1 = sal.cpu().numpy().copy()
+    tiny.ctx.saliency(r, sal)
+    s2 = sal.cpu().numpy()
+    rc, msg = tiny.ctx.last_error()
+    assert rc == moe.OK, msg
+    objs = {int(e): tiny.host_object(0, int(e)) for e in np.unique(ids)}
+    ref = oracle.saliency(x, ids, w, objs, wl.n_experts, wl.hidden, wl.inter)
+    used = np.unique(ids)
+    np.testing.assert_allclose(s1[used], ref[used], rtol=2e-3)
+    assert np.all(s1[np.setdiff1d(np.arange(wl.n_experts), used)] == 0.0)
+    np.testing.assert_array_equal(s2, 2.0 * s1)

@@ -68,6 +68,24 @@ def test_prefill_2048(layer, path):
     check_y(y[toks], layer.oracle_y(0, x, ids, w, toks))
 
 
+@pytest.mark.parametrize("T", [1, 8])
+def test_saliency_full_size(layer, T):
+    wl = synth.WORKLOADS["decode_b1"]
+    x, ids, w, y = _step(layer, wl, T, 21 + T)
+    r = layer.ctx.route(0, to_dev(synth.layer_inputs(wl, 0, 21 + T, tokens=T)[0]))
+    layer.ctx.forward(0, to_dev(x), r)
+    sal = torch.zeros(wl.n_experts, dtype=torch.float64, device="cuda")
+    layer.ctx.saliency(r, sal)
+    rc, msg = layer.ctx.last_error()
+    assert rc == moe.OK, msg
+    s = sal.cpu().numpy()
+    objs = {int(e): layer.host_object(0, int(e)) for e in np.unique(ids)}
+    ref = oracle.saliency(x, ids, w, objs, wl.n_experts, wl.hidden, wl.inter)
+    used = np.unique(ids)
+    np.testing.assert_allclose(s[used], ref[used], rtol=2e-3)
+    assert np.all(s[np.setdiff1d(np.arange(wl.n_experts), used)] == 0.0)
+
+
 def test_unmapped_expert_reports_eslot(layer):
     wl = synth.WORKLOADS["decode_b1"]
     logits, _ = synth.layer_inputs(wl, 0, 11, tokens=1)
