@@ -19,6 +19,7 @@
 #include "fp4_decode.cuh"
 #include "router.cuh"
 #include "slot_layout.cuh"
+#include "residency.h"
 #include "tc_prefill.cuh"
 
 using namespace moe;
@@ -47,6 +48,15 @@ struct moe_fp4_ctx {
     std::vector<ProfRec> prof;         // profiled launches not yet read
     std::vector<cudaEvent_t> ev_free;  // recycled events
     TcPlan tc{};                       // tcgen05 prefill workspace
+    // expert streaming (moe_fp4_stream_experts): LRU clock per slot, two
+    // staging buffers filled on a copy stream, statistics
+    std::vector<uint64_t> slot_last;
+    uint64_t lru_clock = 0;
+    int64_t stream_stats[3] = {0, 0, 0};   // hits, misses, bytes copied
+    uint8_t* d_stage2[2] = {nullptr, nullptr};
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t st_ready[2] = {nullptr, nullptr}, st_free[2] = {nullptr, nullptr};
+    unsigned ring = 0;
     std::string host_msg;
     moe_fp4_status host_status = MOE_FP4_OK;
 };
@@ -347,6 +357,12 @@ void moe_fp4_destroy(moe_fp4_ctx* c) {
     cudaFree(c->d_h);
     cudaFree(c->d_o);
     cudaFree(c->d_norm);
+    for (int b = 0; b < 2; ++b) {
+        if (c->d_stage2[b]) cudaFree(c->d_stage2[b]);
+        if (c->st_ready[b]) cudaEventDestroy(c->st_ready[b]);
+        if (c->st_free[b]) cudaEventDestroy(c->st_free[b]);
+    }
+    if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
     cudaFree(c->d_err);
     cudaFree(c->d_ticket);
     tc_plan_destroy(&c->tc);
@@ -416,6 +432,83 @@ moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx* c, int layer, int expert, i
     if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: launch");
     c->h_table[idx] = slot;
     c->slot_owner[slot] = idx;
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_stream_experts(moe_fp4_ctx* c, int layer, const int32_t* experts, int n,
+                                      const uint8_t* const* objects, int32_t* slots_out, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || n < 0 || (n > 0 && !experts))
+        return host_fail(c, MOE_FP4_EINVAL, "stream_experts: layer %d / n %d / experts", layer, n);
+    if (n > g.n_slots)
+        return host_fail(c, MOE_FP4_EINVAL, "stream_experts: %d experts exceed the %d slots", n, g.n_slots);
+    std::vector<int64_t> keys(n);
+    std::vector<uint8_t> seen(g.n_experts, 0);
+    for (int i = 0; i < n; ++i) {
+        const int e = experts[i];
+        if (e < 0 || e >= g.n_experts || seen[e])
+            return host_fail(c, MOE_FP4_EINVAL, "stream_experts: expert %d out of range or repeated", e);
+        seen[e] = 1;
+        keys[i] = static_cast<int64_t>(layer) * g.n_experts + e;
+        if (c->h_table[keys[i]] < 0 && (!objects || !objects[i]))
+            return host_fail(c, MOE_FP4_EINVAL, "stream_experts: expert %d is not resident and has no object", e);
+    }
+    if (n == 0) return MOE_FP4_OK;
+    cudaSetDevice(c->device);
+    cudaError_t e;
+    if (!c->copy_stream) {   // first use: staging buffers, copy stream, events
+        for (int b = 0; b < 2; ++b) {
+            if ((e = cudaMalloc(&c->d_stage2[b], c->slot_bytes)) != cudaSuccess)
+                return host_fail(c, MOE_FP4_ENOMEM, "stream_experts: staging allocation failed");
+            if ((e = cudaEventCreateWithFlags(&c->st_ready[b], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&c->st_free[b], cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(c, e, "stream_experts: events");
+        }
+        if ((e = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(c, e, "stream_experts: copy stream");
+    }
+    if (c->slot_last.size() != static_cast<size_t>(g.n_slots)) c->slot_last.assign(g.n_slots, 0);
+    std::vector<int32_t> slot(n);
+    std::vector<uint8_t> hit(n);
+    std::vector<int64_t> evicted(n);
+    if (!lru_plan(c->slot_owner.data(), c->h_table.data(), c->slot_last.data(), g.n_slots, ++c->lru_clock,
+                  keys.data(), n, slot.data(), hit.data(), evicted.data()))
+        return host_fail(c, MOE_FP4_EINVAL, "stream_experts: no slot plan");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t threads = 3 * static_cast<size_t>(g.inter) * g.hidden / 16;   // code chunks + scale bytes
+    for (int i = 0; i < n; ++i) {
+        if (hit[i]) {
+            ++c->stream_stats[0];
+            continue;
+        }
+        const unsigned b = c->ring++ & 1u;
+        // the copy waits until the last relayout that read this staging buffer is done
+        if ((e = cudaStreamWaitEvent(c->copy_stream, c->st_free[b], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(c->d_stage2[b], objects[i], c->slot_bytes, cudaMemcpyDefault, c->copy_stream)) !=
+                cudaSuccess ||
+            (e = cudaEventRecord(c->st_ready[b], c->copy_stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(s, c->st_ready[b], 0)) != cudaSuccess)
+            return cuda_fail(c, e, "stream_experts: copy");
+        if (evicted[i] >= 0 &&
+            (e = cudaMemsetAsync(c->d_table + evicted[i], 0xFF, sizeof(int32_t), s)) != cudaSuccess)
+            return cuda_fail(c, e, "stream_experts: evict");
+        load_slot_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
+            c->d_stage2[b], c->arena + static_cast<size_t>(slot[i]) * c->slot_bytes, c->lay, c->d_table,
+            static_cast<int>(keys[i]), slot[i], c->d_err);
+        if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaEventRecord(c->st_free[b], s)) != cudaSuccess)
+            return cuda_fail(c, e, "stream_experts: relayout");
+        ++c->stream_stats[1];
+        c->stream_stats[2] += static_cast<int64_t>(c->slot_bytes);
+    }
+    if (slots_out)
+        for (int i = 0; i < n; ++i) slots_out[i] = slot[i];
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_residency_stats(moe_fp4_ctx* c, int64_t* stats) {
+    if (!c || !stats) return MOE_FP4_EINVAL;
+    for (int i = 0; i < 3; ++i) stats[i] = c->stream_stats[i];
     return MOE_FP4_OK;
 }
 

@@ -24,7 +24,7 @@ OPT_PATH, OPT_PROFILE = 1, 2
 # every symbol include/moe_fp4.h declares
 EXPORTS = ("moe_fp4_slot_bytes", "moe_fp4_create", "moe_fp4_destroy", "moe_fp4_arena",
            "moe_fp4_set_option", "moe_fp4_profile_read", "moe_fp4_load_expert_slot", "moe_fp4_route",
-           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency")
+           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency", "moe_fp4_stream_experts", "moe_fp4_residency_stats")
 
 
 class MoeError(RuntimeError):
@@ -71,6 +71,10 @@ def load(path: str = LIB_PATH):
         L.moe_fp4_forward.argtypes = [P, I32, P, I32, P, P, P, P, P, P, P, P]
         L.moe_fp4_saliency.restype = I32
         L.moe_fp4_saliency.argtypes = [P, I32, P, P, P, P, P]
+        L.moe_fp4_stream_experts.restype = I32
+        L.moe_fp4_stream_experts.argtypes = [P, I32, P, I32, P, P, P]
+        L.moe_fp4_residency_stats.restype = I32
+        L.moe_fp4_residency_stats.argtypes = [P, P]
         L.moe_fp4_last_error.restype = I32
         L.moe_fp4_last_error.argtypes = [P, ctypes.c_char_p, SZ]
         L.moe_fp4_forward_noalloc.restype = I32
@@ -237,6 +241,26 @@ class Context:
         self._check(rc, "forward")
         return y
 
+
+    def stream_experts(self, layer: int, experts, objects, stream=None) -> list[int]:
+        """Make the listed distinct experts of ``layer`` resident (LRU slots).
+        ``objects``: per expert a contiguous checkpoint-layout object (pinned
+        host or device uint8 tensor, or numpy array), or None if resident.
+        Returns the slot of each expert."""
+        n = len(experts)
+        ids = (ctypes.c_int32 * n)(*[int(e) for e in experts])
+        ptrs = (ctypes.c_void_p * n)(*[(_data_ptr(o) if o is not None else None) for o in objects])
+        slots = (ctypes.c_int32 * n)()
+        rc = self.lib.moe_fp4_stream_experts(self.h, layer, ids, n, ptrs, slots, _stream(stream))
+        self._check(rc, "stream_experts")
+        return list(slots)
+
+    def residency_stats(self) -> tuple[int, int, int]:
+        """(hits, misses, bytes copied) of stream_experts since create."""
+        out = (ctypes.c_int64 * 3)()
+        rc = self.lib.moe_fp4_residency_stats(self.h, out)
+        self._check(rc, "residency_stats")
+        return out[0], out[1], out[2]
 
     def saliency(self, r: Routing, sal: torch.Tensor, stream=None) -> torch.Tensor:
         """Accumulate per-expert saliency (fp64 [E] device tensor) of the last

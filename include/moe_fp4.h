@@ -78,14 +78,22 @@ enum {
  * V4.1 shape 18,800,640 (10100.com article, section "moe专家的容量瓶颈").
  * Returns 0 for an invalid config.
  *
- * Slot layout (offsets from the slot base, all multiples of 128 bytes for
- * the V4.1 shape): w1 codes [I, H/2] at 0, w3 codes at I*H/2, w2 codes
- * [H, I/2] at I*H, then s1 [I, H/32], s3 [I, H/32], s2 [H, I/32] scales:
- * codes first, scales after, as the article stores the expert object
- * (section "SSD读取性能").  Inside the slot each 32-bit word of codes is
- * re-encoded by moe_fp4_load_expert_slot (the eight sign bits are moved so
- * that the in-register decoder of csrc/fp4_decode.cuh needs fewer
- * instructions; magnitudes stay in place); scales are stored as is.
+ * The checkpoint stores an expert as codes first, scales after (w1, w3, w2
+ * codes, then s1, s3, s2; the article's section "SSD读取性能"); the loaders
+ * take that layout.  Inside a slot the same bytes are rearranged so that the
+ * kernels stream one contiguous, 16-byte-aligned range per unit of work:
+ *  up blocks, for each 16-row tile rt of W1/W3 and each K block f of KBu
+ *  (256 when it divides H, else 128) columns, in order (rt, f):
+ *      [w1 16 rows x KBu/2][w3 16 rows x KBu/2][s1 16 x KBu/32][s3 16 x KBu/32]
+ *  then down blocks, for each 16-row tile of W2 and each K block of KBd
+ *  (256 when it divides I, else 128):  [w2 16 rows x KBd/2][s2 16 x KBd/32]
+ * so one 16-row tile of w1+w3 over all of H (87,040 bytes for V4.1) and 32
+ * rows of w2 over all of I (39,168 bytes) are each contiguous.  In code rows
+ * of 128-byte multiples the 16-byte chunk q of row r sits at
+ * q ^ ((r & 7) ^ ((r & 1) << 2)) (bank-conflict-free loads), and each 32-bit
+ * code word is re-encoded (the eight sign bits move so that the in-register
+ * decoder of csrc/fp4_decode.cuh needs fewer instructions; magnitudes stay in
+ * place).  Scale bytes are stored as they are.  The total is unchanged.
  */
 size_t moe_fp4_slot_bytes(const moe_fp4_config *cfg);
 
@@ -145,6 +153,36 @@ moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx *ctx, int layer, int expert,
                                         const uint8_t *w3, const uint8_t *w3_scale,
                                         const uint8_t *w2, const uint8_t *w2_scale,
                                         void *stream);
+
+/*
+ * Stream experts into a smaller arena (the hot-expert arena of 10100.com
+ * article 151357339, section "方案一": a fixed set of slots filled on demand,
+ * the least recently used expert making room).  For the n distinct experts of
+ * `layer` that one forward needs, experts already resident are hits; each
+ * miss takes the lowest-numbered free slot, else the slot whose last request
+ * is oldest among those this request does not use (lowest number on ties),
+ * evicting its expert (csrc/residency.h).  A miss's object is copied on an
+ * internal copy stream into one of two staging buffers, which overlaps with
+ * the relayout of the previous miss on `stream`; the relayout (as
+ * moe_fp4_load_expert_slot) and the slot-table update run on `stream`, so a
+ * forward issued after this call on `stream` sees them.
+ *  experts  int32 [n] host: distinct expert ids of `layer`, n <= n_slots.
+ *  objects  host array [n] of pointers to contiguous expert objects in
+ *           checkpoint layout (w1, w3, w2 codes, s1, s3, s2 scales; pinned
+ *           host memory for the copy to be asynchronous, or device memory);
+ *           objects[i] may be NULL only when experts[i] is resident.
+ *  slots_out int32 [n] host or NULL: the slot of each expert after the call.
+ * Work already queued on `stream` that reads an evicted slot is not affected
+ * (the relayout runs after it); work on other streams must be ordered by the
+ * caller.  Errors: EINVAL (before any change: bad layer, ids, repeated id,
+ * n > n_slots, missing object), ENOMEM, ECUDA.
+ */
+moe_fp4_status moe_fp4_stream_experts(moe_fp4_ctx *ctx, int layer, const int32_t *experts, int n,
+                                      const uint8_t *const *objects, int32_t *slots_out, void *stream);
+
+/* Streaming counters since create: stats[0] hits, [1] misses, [2] bytes
+ * copied by moe_fp4_stream_experts.  Errors: EINVAL (NULL). */
+moe_fp4_status moe_fp4_residency_stats(moe_fp4_ctx *ctx, int64_t *stats);
 
 /*
  * Route T tokens of one layer (one kernel launch).
