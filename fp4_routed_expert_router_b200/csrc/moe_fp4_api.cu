@@ -37,6 +37,7 @@ struct moe_fp4_ctx {
     uint16_t* d_h = nullptr;           // [max_tokens*k, I] bf16
     float* d_o = nullptr;              // [max_tokens*k, H] fp32
     float* d_norm = nullptr;           // [max_tokens*k] fp32 (saliency)
+    int32_t* d_grp = nullptr;          // expert_outputs grouping: counts [E], offsets [E+1], perm [max_tokens*k]
     int* d_err = nullptr;              // error word [4]
     unsigned int* d_ticket = nullptr;  // route kernel ticket
     std::vector<int32_t> h_table;      // host mirror of d_table
@@ -322,6 +323,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaMalloc(&c->d_h, sizeof(uint16_t) * ent * I) != cudaSuccess ||
         cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
         cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
+        cudaMalloc(&c->d_grp, sizeof(int32_t) * (2 * static_cast<size_t>(cfg->n_experts) + 1 + ent)) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
         cudaGetLastError();
@@ -357,6 +359,7 @@ void moe_fp4_destroy(moe_fp4_ctx* c) {
     cudaFree(c->d_h);
     cudaFree(c->d_o);
     cudaFree(c->d_norm);
+    cudaFree(c->d_grp);
     for (int b = 0; b < 2; ++b) {
         if (c->d_stage2[b]) cudaFree(c->d_stage2[b]);
         if (c->st_ready[b]) cudaEventDestroy(c->st_ready[b]);
@@ -571,6 +574,52 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
                  static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
     if (e != cudaSuccess) return cuda_fail(c, e, "forward: combine launch");
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_expert_outputs(moe_fp4_ctx* c, int layer, const uint16_t* x, int n, const int32_t* experts,
+                                      float* o, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || n < 0 || n > g.max_tokens * g.top_k)
+        return host_fail(c, MOE_FP4_EINVAL, "expert_outputs: layer %d / n %d out of range", layer, n);
+    if (n == 0) return MOE_FP4_OK;
+    if (!x || !experts || !o) return host_fail(c, MOE_FP4_EINVAL, "expert_outputs: NULL argument");
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(o) & 15))
+        return host_fail(c, MOE_FP4_EINVAL, "expert_outputs: x and o must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int H = g.hidden, I = g.inter, E = g.n_experts;
+    int32_t* counts = c->d_grp;
+    int32_t* offsets = counts + E;
+    int32_t* perm = offsets + E + 1;
+    // group the n entries by expert (one CTA; entries with an id outside [0, E) latch EINVAL)
+    RouteArgs ra{nullptr, nullptr, n, E, 1, const_cast<int32_t*>(experts), nullptr, counts, offsets, perm,
+                 c->d_ticket, c->d_err};
+    cudaError_t e = launch_k(c, "group", group_kernel, dim3(1), dim3(kRouteWarps * 32),
+                             sizeof(int) * kRouteWarps * E, s, ra);
+    if (e != cudaSuccess) return cuda_fail(c, e, "expert_outputs: group launch");
+    GemvArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, 1, H, I, x, offsets, perm, c->d_h, o, c->d_err};
+    const bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && 4LL * n >= 3LL * E);
+    e = use_tc ? tc_forward(c, a, c->lay, n, s)
+               : decode_forward(c, a, c->lay, n < E ? n : E, c->sm_count, c->smem_optin, s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "expert_outputs: expert FFN launch");
+    return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_combine(moe_fp4_ctx* c, int T, const float* o, const float* weights, const uint16_t* x,
+                               float* y, uint16_t* x_out, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (T < 0 || T > g.max_tokens) return host_fail(c, MOE_FP4_EINVAL, "combine: T %d out of range", T);
+    if (T == 0) return MOE_FP4_OK;
+    if (!o || !weights || !y || (x_out && !x)) return host_fail(c, MOE_FP4_EINVAL, "combine: NULL argument");
+    if ((reinterpret_cast<uintptr_t>(o) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
+        (x_out && ((reinterpret_cast<uintptr_t>(x) & 7) || (reinterpret_cast<uintptr_t>(x_out) & 7))))
+        return host_fail(c, MOE_FP4_EINVAL, "combine: o and y must be 16-byte aligned, x and x_out 8-byte");
+    const int n4 = T * (g.hidden / 4);
+    cudaError_t e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0,
+                             static_cast<cudaStream_t>(stream), o, weights, x, T, g.hidden, g.top_k, y, x_out);
+    if (e != cudaSuccess) return cuda_fail(c, e, "combine: launch");
     return MOE_FP4_OK;
 }
 

@@ -165,6 +165,15 @@ __device__ void group_entries(const RouteArgs& a, int* hist) {
     }
 }
 
+// Grouping alone: the a.T given expert ids (a.k = 1) grouped by expert, as
+// the route kernels group their selections (the expert-parallel owner side).
+__global__ void __launch_bounds__(kRouteWarps * 32) group_kernel(RouteArgs a) {
+    extern __shared__ int smem_hist[];
+    pdl_wait();
+    group_entries(a, smem_hist);
+    pdl_trigger();
+}
+
 template <int NI>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     extern __shared__ int smem_hist[];

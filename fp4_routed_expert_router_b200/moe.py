@@ -24,7 +24,7 @@ OPT_PATH, OPT_PROFILE = 1, 2
 # every symbol include/moe_fp4.h declares
 EXPORTS = ("moe_fp4_slot_bytes", "moe_fp4_create", "moe_fp4_destroy", "moe_fp4_arena",
            "moe_fp4_set_option", "moe_fp4_profile_read", "moe_fp4_load_expert_slot", "moe_fp4_route",
-           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency", "moe_fp4_stream_experts", "moe_fp4_residency_stats")
+           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency", "moe_fp4_stream_experts", "moe_fp4_residency_stats", "moe_fp4_expert_outputs", "moe_fp4_combine")
 
 
 class MoeError(RuntimeError):
@@ -75,6 +75,10 @@ def load(path: str = LIB_PATH):
         L.moe_fp4_stream_experts.argtypes = [P, I32, P, I32, P, P, P]
         L.moe_fp4_residency_stats.restype = I32
         L.moe_fp4_residency_stats.argtypes = [P, P]
+        L.moe_fp4_expert_outputs.restype = I32
+        L.moe_fp4_expert_outputs.argtypes = [P, I32, P, I32, P, P, P]
+        L.moe_fp4_combine.restype = I32
+        L.moe_fp4_combine.argtypes = [P, I32, P, P, P, P, P, P]
         L.moe_fp4_last_error.restype = I32
         L.moe_fp4_last_error.argtypes = [P, ctypes.c_char_p, SZ]
         L.moe_fp4_forward_noalloc.restype = I32
@@ -241,6 +245,27 @@ class Context:
         self._check(rc, "forward")
         return y
 
+
+    def expert_outputs(self, layer: int, x: torch.Tensor, experts: torch.Tensor, o: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+        """o[i] = expert experts[i] applied to x[i] (fp32 [n, H]); x bf16 bits [n, H]."""
+        n = x.shape[0]
+        if o is None:
+            o = torch.empty((n, self.cfg.hidden), dtype=torch.float32, device=x.device)
+        rc = self.lib.moe_fp4_expert_outputs(self.h, layer, _ptr(x), n, _ptr(experts), _ptr(o), _stream(stream))
+        self._check(rc, "expert_outputs")
+        return o
+
+    def combine(self, o: torch.Tensor, weights: torch.Tensor, x: torch.Tensor | None = None,
+                y: torch.Tensor | None = None, x_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """y[t] = sum_j weights[t, j] * o[t*k + j] (+ x_out = bf16(x + y))."""
+        T = weights.shape[0]
+        if y is None:
+            y = torch.empty((T, self.cfg.hidden), dtype=torch.float32, device=o.device)
+        rc = self.lib.moe_fp4_combine(self.h, T, _ptr(o), _ptr(weights), _ptr(x), _ptr(y), _ptr(x_out),
+                                      _stream(stream))
+        self._check(rc, "combine")
+        return y
 
     def stream_experts(self, layer: int, experts, objects, stream=None) -> list[int]:
         """Make the listed distinct experts of ``layer`` resident (LRU slots).

@@ -223,6 +223,37 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, i
                                const int32_t *perm, float *y, uint16_t *x_out, void *stream);
 
 /*
+ * The expert FFN for an arbitrary list of (row, expert) pairs of `layer`:
+ *   o[i] = expert_{experts[i]}(x[i])   (fp32 [n, H], no router weight)
+ * This is the work an expert-parallel rank does for the entries other ranks
+ * dispatch to the experts it holds (moe_fp4_forward = route + this for every
+ * (token, selected expert) pair + moe_fp4_combine).  The entries are grouped
+ * by expert with the route kernels' stable grouping, then run on the GEMV
+ * path, or on the tcgen05 path when 4n >= 3E (or as MOE_FP4_OPT_PATH forces).
+ * Entries are processed in the same per-expert order as moe_fp4_forward
+ * processes (token, slot) entries, so listing a forward's entries in
+ * (token, slot) order reproduces its per-entry outputs bit for bit.
+ *  x        bf16 [n, H] device, 16-byte aligned (row i goes with experts[i]).
+ *  experts  int32 [n] device; an id outside [0, E) latches EINVAL and its
+ *           row of o is left unwritten.
+ *  o        fp32 [n, H] device out, 16-byte aligned.
+ * n <= max_tokens * top_k; uses the context's workspace like forward.
+ * Errors: EINVAL, ECUDA; unmapped experts latch ESLOT (their rows are zero).
+ */
+moe_fp4_status moe_fp4_expert_outputs(moe_fp4_ctx *ctx, int layer, const uint16_t *x, int n,
+                                      const int32_t *experts, float *o, void *stream);
+
+/*
+ * The combine step alone: y[t] = sum over j < k of weights[t, j] * o[t*k + j]
+ * (fixed j order, fp32), and x_out = bf16_rne(x + y) when x_out is not NULL
+ * (x_out may alias x).  o fp32 [T*k, H] and y fp32 [T, H] 16-byte aligned;
+ * x, x_out bf16 [T, H] 8-byte aligned.  T <= max_tokens.  Errors: EINVAL,
+ * ECUDA.
+ */
+moe_fp4_status moe_fp4_combine(moe_fp4_ctx *ctx, int T, const float *o, const float *weights,
+                               const uint16_t *x, float *y, uint16_t *x_out, void *stream);
+
+/*
  * Expert saliency of the last forward (10100.com article 151357339, section
  * "选哪些专家：频率 vs Saliency": router weight times the L2 norm of the
  * expert's output, summed over a corpus, used to rank experts for pruning):
