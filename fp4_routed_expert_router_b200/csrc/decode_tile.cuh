@@ -200,7 +200,10 @@ __global__ void __launch_bounds__((RB * KS + 1) * 32, 1) gemv_tile_kernel(GemvAr
         if (!mbar_wait(&full[st], (i / p.stages) & 1, abort_flag) && lane == 0)
             latch_error(a.err, ERR_ETIMEOUT, i, UP ? KID_UP : KID_DOWN);
         const uint8_t* stg = smem + p.off_stage + static_cast<size_t>(st) * p.stage_bytes;
+        // two accumulators per matrix (even / odd MMA of each code word) halve
+        // the chain of dependent mma.sync; summed once per item
         float d1[4] = {0.f, 0.f, 0.f, 0.f}, d3[4] = {0.f, 0.f, 0.f, 0.f};
+        float e1[4] = {0.f, 0.f, 0.f, 0.f}, e3[4] = {0.f, 0.f, 0.f, 0.f};
         if (slot >= 0) {
 #pragma unroll
             for (int j = 0; j < CPW; ++j) {
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__((RB * KS + 1) * 32, 1) gemv_tile_kernel(GemvAr
                     fp4_decode8(word(Aa, w), La, oa);
                     fp4_decode8(word(Ab, w), Lb, ob);
                     mma_bf16_16816(d1, oa[0], ob[0], oa[1], ob[1], word(X[j][w], 0), word(X[j][w], 1));
-                    mma_bf16_16816(d1, oa[2], ob[2], oa[3], ob[3], word(X[j][w], 2), word(X[j][w], 3));
+                    mma_bf16_16816(e1, oa[2], ob[2], oa[3], ob[3], word(X[j][w], 2), word(X[j][w], 3));
                 }
                 if (UP) {
                     const uint4 Ca = *reinterpret_cast<const uint4*>(ra + 16 * rbb);
@@ -233,9 +236,14 @@ __global__ void __launch_bounds__((RB * KS + 1) * 32, 1) gemv_tile_kernel(GemvAr
                         fp4_decode8(word(Ca, w), Lc, pa);
                         fp4_decode8(word(Cb, w), Ld, pb);
                         mma_bf16_16816(d3, pa[0], pb[0], pa[1], pb[1], word(X[j][w], 0), word(X[j][w], 1));
-                        mma_bf16_16816(d3, pa[2], pb[2], pa[3], pb[3], word(X[j][w], 2), word(X[j][w], 3));
+                        mma_bf16_16816(e3, pa[2], pb[2], pa[3], pb[3], word(X[j][w], 2), word(X[j][w], 3));
                     }
                 }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                d1[q] += e1[q];
+                d3[q] += e3[q];
             }
         } else if (tid == 0) {
             latch_error(a.err, ERR_ESLOT, act_e[ai], UP ? KID_UP : KID_DOWN);
