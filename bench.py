@@ -8,8 +8,10 @@ One step = one pass of the whole path (route + w1/w3 GEMM + SwiGLU + w2 GEMM
 layer (hidden 5120, inter 2304, 384 experts resident in the arena, top-6).
 The JSON line's value is the --workload (default decode batch 1); the other
 workloads of the same layer (decode batch 64, prefill 2048 tokens) are timed
-on the same arena right after it, then the 40-layer stack (batch 1 and 8, its
-own 115.8 GB arena), all reported under "workloads".
+on the same arena right after it, then decode batch 1 with only 25 % of the
+experts resident and the rest streamed from pinned host memory, then the
+40-layer stack (batch 1 and 8, its own 115.8 GB arena), all reported under
+"workloads".
 Inputs are resident in HBM when a timed step starts; L2 is flushed between
 timed steps (a 2x L2-sized write), so expert bytes really come from HBM.
 Rank 0 prints one JSON line.  Under torchrun each rank runs an independent
@@ -481,6 +483,62 @@ def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
     return out
 
 
+def run_streaming(wl, local, resident_frac, steps, warmup):
+    """Decode with an arena smaller than the layer: only resident_frac of the
+    experts have slots, the rest stream in on demand from pinned host memory
+    (moe_fp4_stream_experts, least recently used slots).  One step = route ->
+    chosen ids to the host -> stream the misses -> forward, for one token; the
+    host takes part in every step, so the time is wall-clock around the step
+    with the device synchronised at both ends."""
+    import torch
+    from fp4_routed_expert_router_b200 import moe
+    dev = torch.device("cuda", local)
+    E = wl.n_experts
+    n_slots = max(wl.top_k, int(round(resident_frac * E)))
+    ctx = moe.Context(wl.hidden, wl.inter, E, wl.top_k, 1, n_slots, 8, device=local)
+    staging = torch.empty(wl.expert_bytes, dtype=torch.uint8, device=dev)
+    host = []
+    for e in range(E):   # the expert store: every expert's checkpoint object in pinned host memory
+        moe.synth_fill_expert(staging, wl.seed, 0, e, wl.hidden, wl.inter, wl.scale_lo, wl.scale_hi)
+        h = torch.empty(wl.expert_bytes, dtype=torch.uint8, pin_memory=True)
+        h.copy_(staging)
+        host.append(h)
+    del staging
+    T = wl.tokens
+    npool = 64
+    pool_x = [torch.from_numpy(synth.gen_x(wl.seed, T, wl.hidden, 50_000 + i).view(np.int16)).to(dev)
+              for i in range(npool)]
+    pool_l = [torch.from_numpy(synth.layer_inputs(wl, 0, 50_000 + i)[0]).to(dev) for i in range(npool)]
+    r = ctx.alloc_routing(T)
+    y = torch.empty((T, wl.hidden), dtype=torch.float32, device=dev)
+
+    def step(i):
+        ctx.route(0, pool_l[i % npool], out=r)
+        need = sorted({int(e) for e in r.ids.reshape(-1).tolist()})
+        ctx.stream_experts(0, need, [host[e] for e in need])
+        ctx.forward(0, pool_x[i % npool], r, y=y)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    h0 = ctx.residency_stats()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        step(warmup + i)
+    torch.cuda.synchronize()
+    sec = time.perf_counter() - t0
+    h1 = ctx.residency_stats()
+    rc, msg = ctx.last_error()
+    assert rc == moe.OK, msg
+    hits, misses, nbytes = (h1[j] - h0[j] for j in range(3))
+    ctx.close()
+    return {"steps": steps, "tok_s": T * steps / sec, "ms_per_step": 1e3 * sec / steps,
+            "resident_slots": n_slots, "resident_fraction": n_slots / E,
+            "hit_rate": hits / max(1, hits + misses), "misses_per_step": misses / steps,
+            "h2d_gbs": nbytes / sec / 1e9, "timing": "wall clock, host in the loop (ids read back every step)",
+            "expert_store": "pinned host memory, checkpoint layout"}
+
+
 def roofline(wl, res, peaks, peak_src):
     """Roofline of the step's dominant kernel, the w1/w3 one (gemv_up or
     tc_up).  Algorithmic bytes = active experts x w1/w3 codes + scales;
@@ -565,6 +623,9 @@ def run_ours(args, wl):
         r2 = bench.run(w2, steps2, max(3, min(args.warmup, 5)), not args.no_graph, 8, clocks=True)
         sec[n] = {"steps": steps2, **summary(w2, r2, steps2, world, peaks, peak_src), "clocks": r2["clocks"]}
 
+    if not args.only and wl.name == "decode_b1":
+        sec["stream_decode_b1_25pct"] = run_streaming(wl, local, 0.25, min(args.steps, 100),
+                                                      max(3, min(args.warmup, 50)))
     if not args.only and wl.n_experts == synth.WORKLOADS["stack40_b1"].n_experts:
         bench.ctx.close()
         bench.ctx = None
