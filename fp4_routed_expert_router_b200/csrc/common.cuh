@@ -34,16 +34,6 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
-// 16-byte streaming load that is not kept in L1 (weights are read once).
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint4 ldg_cached(const void* p) {
-    return __ldg(reinterpret_cast<const uint4*>(p));
-}
 // Coherent L2 load for data written earlier in the same grid (no L1).
 __device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
 

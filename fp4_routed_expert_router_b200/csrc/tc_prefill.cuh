@@ -13,27 +13,30 @@
 //         slot block g -- so silu(a1) * a3 pairs lanes l and l + 16 of one
 //         warp (a shuffle, no shared memory);
 //   down  128 output rows, lane r = row r.
-// Both GEMMs therefore run the same pipeline on a 128 x 64 bf16 A tile per
-// K step.  One persistent CTA per SM, warp roles:
+// Both GEMMs therefore run the same pipeline on a 128 x 128 bf16 A tile per
+// stage (128 K, two 128-byte swizzle atoms).  One persistent CTA per SM, warp
+// roles:
 //   warps 0-15   dequantisers: warp w works in TMEM lane group w % 4 and
-//                takes every fourth K step (residue w / 4); each thread
-//                decodes its row's 64 codes of the step (two 32-K chunks) from
-//                the staged FP4 blocks (exact E2M1 x 2^(s-127) -> bf16,
-//                fp4_decode.cuh) and writes them to the step's A stage in
-//                TMEM with tcgen05.st (lane = row, two bf16 per column).
+//                decodes 32-K chunk w / 4 of every stage: each thread takes
+//                its row's 32 codes from the staged FP4 blocks (exact E2M1 x
+//                2^(s-127) -> bf16, fp4_decode.cuh) and writes them to the
+//                stage's A columns in TMEM with tcgen05.st (lane = row, two
+//                bf16 per column).
 //   warps 16-19  epilogue: tcgen05.ld of the finished accumulator (double
 //                buffered), SwiGLU -> h (bf16) or o (fp32, scattered back to
 //                token-expert order), overlapping the next item's MMAs.
-//   warp 20      B producer: TMA tensor loads of the step's 16-row boxes of
+//   warp 20      B producer: TMA tensor loads of the stage's 16-row boxes of
 //                gathered token rows (x grouped by expert, or h), 128-byte
 //                swizzle, into shared memory.
 //   warp 21      code producer: cp.async.bulk of the item's slot blocks (all
-//                of its rows for one block's K = four steps) into a ring.
+//                of its rows for one block's K = two stages) into a ring.
 //   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A from
-//                TMEM and B from shared memory (fp32 accumulate in TMEM), four
-//                K=16 instructions per step; tcgen05.commit frees the stage
-//                and, after the last step, hands the accumulator over.
-// Every party walks the same sequence of steps and items, so each parity wait
+//                TMEM and B from shared memory (fp32 accumulate in TMEM), eight
+//                K=16 instructions per stage; tcgen05.commit frees the stage
+//                and, after the last stage, hands the accumulator over.
+// A stage is "full" when all 16 dequant warps have arrived and the B bytes
+// have landed (one mbarrier: 16 arrivals + the producer's expect-tx).
+// Every party walks the same sequence of stages and items, so each parity wait
 // is unambiguous; every wait is bounded and the first one that gives up
 // aborts the CTA's remaining waits (MOE_FP4_ETIMEOUT), after producers have
 // let their copies in flight land.
@@ -88,16 +91,8 @@ __device__ __forceinline__ uint32_t umma_idesc_bf16(int m, int n) {
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Same, with A read from tensor memory (lane = row, two bf16 per column).
+// One tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128) with A read from
+// tensor memory (lane = row, two bf16 per column) and B from shared memory.
 __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
     asm volatile(
@@ -114,7 +109,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
     asm volatile(
@@ -132,18 +126,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) 
             taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

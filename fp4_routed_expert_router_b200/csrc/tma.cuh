@@ -87,21 +87,4 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     return true;
 }
 
-// Bounded wait until *counter > value (shared memory, written by another warp
-// of the CTA); same abort protocol as mbar_wait.
-__device__ __forceinline__ bool wait_counter_above(volatile int* counter, int value, volatile int* abort,
-                                                   uint64_t timeout_ns = 1000000000ull) {
-    if (*counter > value) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (*counter <= value) {
-        if (*abort) return false;
-        if (global_timer_ns() - t0 > timeout_ns) {
-            *abort = 1;
-            return false;
-        }
-        __nanosleep(64);
-    }
-    return true;
-}
-
 }  // namespace moe
