@@ -237,7 +237,7 @@ bool decode_shape_ok(const SlotLayout& L) {
 
 cudaError_t allow_decode_smem_all(int bytes) {
     cudaError_t e = cudaSuccess, r;
-    if ((r = allow_tile_smem<true, 1, 10, 4>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_tile_smem<true, 1, 8, 5>(bytes)) != cudaSuccess) e = r;
     if ((r = allow_tile_smem<true, 1, 2, 1>(bytes)) != cudaSuccess) e = r;
     if ((r = allow_tile_smem<false, 2, 6, 3>(bytes)) != cudaSuccess) e = r;
     if ((r = allow_tile_smem<false, 2, 1, 1>(bytes)) != cudaSuccess) e = r;
@@ -250,11 +250,11 @@ cudaError_t decode_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& 
                            int smem_limit, cudaStream_t s) {
     if (!decode_shape_ok(L)) return cudaErrorNotSupported;
     const bool big_up = (L.H / 128 == 40), big_down = (L.I / 128 == 18);
-    const TilePlan pu = make_tile_plan(true, L, 1, big_up ? 10 : 2, a.E, active_max, smem_limit);
+    const TilePlan pu = make_tile_plan(true, L, 1, big_up ? 8 : 2, a.E, active_max, smem_limit);
     const TilePlan pd = make_tile_plan(false, L, 2, big_down ? 12 : 2, a.E, active_max, smem_limit);
     if (!pu.stages || !pd.stages) return cudaErrorNotSupported;
     const dim3 grid(static_cast<unsigned>(sm_count));
-    cudaError_t e = big_up ? launch_tile<true, 1, 10, 4>(c, grid, s, a, L, pu)
+    cudaError_t e = big_up ? launch_tile<true, 1, 8, 5>(c, grid, s, a, L, pu)
                            : launch_tile<true, 1, 2, 1>(c, grid, s, a, L, pu);
     if (e != cudaSuccess) return e;
     return big_down ? launch_tile<false, 2, 6, 3>(c, grid, s, a, L, pd)
