@@ -219,11 +219,12 @@ def source_digest(files) -> str:
     return h.hexdigest()[:16]
 
 
-def stored_traffic(kernel: str, workload: str):
+def stored_traffic(kernel: str, workload: str, path: str | None = None):
     """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
-    recorded in profiles/traffic.json for this kernel and workload, or None
-    when there is none or its sources changed since the capture."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    recorded in profiles/traffic.json (or ``path``) for this kernel and
+    workload, or None when there is none or its sources changed since the
+    capture."""
+    p = path or os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
