@@ -29,6 +29,13 @@
  *    moe_fp4_last_error.  No kernel traps; there is no CPU fallback.
  *  - A context is bound to one device; calls must be made with that device
  *    current.  A context is not thread-safe.
+ *
+ * Calls: slot_bytes, create, destroy, arena, set_option, profile_read (the
+ * context); load_expert_slot, stream_experts, residency_stats (the arena);
+ * route, forward, last_error (the layer); expert_outputs, combine (the two
+ * halves of forward, for expert-parallel use); saliency (per-expert
+ * statistic of the last forward); forward_noalloc (forward without any
+ * allocation, library-owned static scratch).
  */
 #ifndef MOE_FP4_H
 #define MOE_FP4_H
@@ -63,7 +70,7 @@ typedef struct {
 
 /* Execution-path override for moe_fp4_set_option(MOE_FP4_OPT_PATH, .). */
 enum {
-    MOE_FP4_PATH_AUTO = 0,  /* grouped GEMV for small batches, tcgen05 GEMM above */
+    MOE_FP4_PATH_AUTO = 0,  /* grouped GEMV while 4*T*k < 3*E, tcgen05 GEMM from there on */
     MOE_FP4_PATH_GEMV = 1,  /* always the register-decoded grouped GEMV */
     MOE_FP4_PATH_TC = 2     /* always the tcgen05 grouped GEMM */
 };
