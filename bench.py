@@ -624,7 +624,7 @@ def run_ours(args, wl):
         r2 = bench.run(w2, steps2, max(3, min(args.warmup, 5)), not args.no_graph, 8, clocks=True)
         sec[n] = {"steps": steps2, **summary(w2, r2, steps2, world, peaks, peak_src), "clocks": r2["clocks"]}
 
-    if not args.only and wl.name == "decode_b1":
+    if not args.only and wl.name == "decode_b1" and world == 1:   # host memory and PCIe are shared by ranks
         sec["stream_decode_b1_25pct"] = run_streaming(wl, local, 0.25, min(args.steps, 100),
                                                       max(3, min(args.warmup, 50)))
     if not args.only and wl.n_experts == synth.WORKLOADS["stack40_b1"].n_experts:
