@@ -70,6 +70,11 @@ def test_null_context_rejected(lib):
     assert lib.moe_fp4_route(None, 0, None, None, 0, None, None, None, None, None, None) == moe.EINVAL
     assert lib.moe_fp4_forward(None, 0, None, 0, None, None, None, None, None, None, None, None) == moe.EINVAL
     assert lib.moe_fp4_last_error(None, None, 0) == moe.EINVAL
+    assert lib.moe_fp4_saliency(None, 0, None, None, None, None, None) == moe.EINVAL
+    assert lib.moe_fp4_stream_experts(None, 0, None, 0, None, None, None) == moe.EINVAL
+    assert lib.moe_fp4_residency_stats(None, None) == moe.EINVAL
+    assert lib.moe_fp4_expert_outputs(None, 0, None, 0, None, None, None) == moe.EINVAL
+    assert lib.moe_fp4_combine(None, 0, None, None, None, None, None, None) == moe.EINVAL
     lib.moe_fp4_destroy(None)
 
 
