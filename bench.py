@@ -63,7 +63,9 @@ def workload_config(wl: synth.Workload, graph: bool) -> dict:
         "logits": f"N(0,1) + Zipf(1.1) bias, alpha {wl.zipf_alpha}",
         "scale_exponents": f"uniform {wl.scale_lo}..{wl.scale_hi}",
         "l2": "flushed between timed steps (2x L2 write)",
-        "launch": "cuda graph of route+forward (PDL chain)" if graph else "eager (PDL chain)",
+        "launch": ("cuda graph of moe_fp4_route_forward" if graph else "eager moe_fp4_route_forward") +
+                  (" (one persistent kernel per step)" if wl.tokens * wl.top_k <= 64 else
+                   " (route kernel, then the expert kernels)"),
         "parallelism": "replicas (one independent layer per GPU)",
     }
 
@@ -278,8 +280,7 @@ class Bench:
         flush = self.flush
 
         def step_launch():
-            ctx.route(0, l_buf, out=routing, stream=stream)
-            ctx.forward(0, x_buf, routing, y=y_buf, stream=stream)
+            ctx.route_forward(0, l_buf, x_buf, out=routing, y=y_buf, stream=stream)
 
         def stage(i):
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
@@ -420,8 +421,8 @@ def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
 
         def step_launch():
             for l in range(L):
-                ctx.route(l, l_buf[l], masks[l], out=routes[l], stream=stream)
-                ctx.forward(l, x_buf, routes[l], y=y_buf, x_out=x_buf, stream=stream)
+                ctx.route_forward(l, l_buf[l], x_buf, keep=masks[l], out=routes[l], y=y_buf, x_out=x_buf,
+                                  stream=stream)
 
         def stage(i):
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
@@ -477,7 +478,7 @@ def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
                         "expert_bytes_per_step": nbytes, "active_experts_per_step": sum(active),
                         "hbm_gbs_step": nbytes / (ms * 1e-3) / 1e9,
                         "hbm_frac_step": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                        "launch": "one cuda graph of 40 x (route + forward)" if graph is not None else "eager",
+                        "launch": "one cuda graph of 40 x moe_fp4_route_forward" if graph is not None else "eager",
                         "clocks": clk.summary()}
         del graph
     ctx.close()
@@ -541,17 +542,25 @@ def run_streaming(wl, local, resident_frac, steps, warmup):
 
 
 def roofline(wl, res, peaks, peak_src):
-    """Roofline of the step's dominant kernel, the w1/w3 one (gemv_up or
-    tc_up).  Algorithmic bytes = active experts x w1/w3 codes + scales;
-    algorithmic FLOPs = 2 GEMMs x 2 H I per token-expert pair.  The bound is
-    the one the arithmetic intensity selects against the measured ridge
-    point; the tensor-core path also reports its fraction of the bf16 peak."""
+    """Roofline of the step's dominant kernel.  Decode batches run the whole
+    layer in one kernel (decode_layer): its algorithmic bytes are every active
+    expert's weights, codes + scales (18,800,640 B each).  Larger batches run
+    the tcgen05 GEMMs; the w1/w3 one (tc_up) dominates: active experts x w1/w3
+    codes + scales.  Algorithmic FLOPs = 2 H I per matrix per token-expert
+    pair.  The bound is the one the arithmetic intensity selects against the
+    measured ridge point; a tensor-core kernel also reports its fraction of
+    the bf16 peak."""
     E, H, I, k, T = wl.n_experts, wl.hidden, wl.inter, wl.top_k, wl.tokens
     avg, act = res["kernel_ms"], res["active"]
-    kern = "tc_up" if "tc_up" in avg else ("gemv_up" if "gemv_up" in avg else max(avg, key=avg.get))
+    if "decode_layer" in avg:
+        kern = "decode_layer"
+        nbytes = act * wl.expert_bytes
+        flops = 6.0 * H * I * T * k
+    else:
+        kern = "tc_up" if "tc_up" in avg else max(avg, key=avg.get)
+        nbytes = act * 2 * (I * H // 2 + I * H // 32)
+        flops = 2.0 * 2.0 * H * I * T * k
     sec = avg[kern] * 1e-3
-    nbytes = act * 2 * (I * H // 2 + I * H // 32)
-    flops = 2.0 * 2.0 * H * I * T * k
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     gbs, tfs = nbytes / sec / 1e9, flops / sec / 1e12
     out_hbm = {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -1,29 +1,19 @@
-// decode_common.cuh -- pieces shared by the decode kernels: arguments, the
-// mma.sync wrapper, the per-scale decode tables, and the combine kernel.
+// decode_common.cuh -- arguments of the expert kernels and the small
+// kernels around them: the router-weighted combine, per-entry output norms
+// and the per-expert saliency.
 //
 // Per active expert e with M_e routed entries the layer needs
 //   a1 = x W1^T, a3 = x W3^T  (W1, W3: [I, H]),  h = bf16(silu(a1) * a3),
-//   o  = h W2^T               (W2: [H, I]),
+//   o  = h W2^T               (W2: [H, I]),       y[t] = sum_j w[t, j] o[t, j]
 // with W = E2M1 * 2^(s-127) (10100.com article 151357339, section
-// "moe专家的容量瓶颈"; SwiGLU is the reading of the unnamed activation).
-// At decode the weights are read once per step and the work is bound by HBM;
-// the decode kernels turn FP4 codes into exact bf16 in registers
-// (fp4_decode.cuh) and let the tensor cores do the multiply-adds through
-// mma.sync.m16n8k16 (bf16 in, fp32 accumulate): one MMA covers 16 weight rows
-// x 16 K x 8 tokens, so up to 8 tokens of an expert share each decoded weight.
-//
-// K order inside an MMA is free as long as A and B agree: lane (g, c) of a
-// warp takes the 32 codes K = kb+32c .. kb+32c+31 of rows g and g+8 (one
-// 16-byte vector and one scale byte each) and uses codes 4i..4i+3 in MMA step
-// i (i = 0..7); its B fragment is x[token g][kb+32c+4i .. +3], so a 16x128
-// weight chunk and a 128-long x slice pair up element for element.
+// "moe专家的容量瓶颈"; SwiGLU is the reading of the unnamed activation, the
+// weighted sum of the expert outputs the reading of the combine).
 #pragma once
 #include "common.cuh"
-#include "fp4_decode.cuh"
 
 namespace moe {
 
-struct GemvArgs {
+struct ExpertArgs {
     const uint8_t* arena;
     size_t slot_bytes;
     const int32_t* slot_table;   // [L][E]
@@ -31,27 +21,9 @@ struct GemvArgs {
     const uint16_t* x;           // [T, H] bf16
     const int32_t* offsets;      // [E+1]
     const int32_t* perm;         // [T*k]
-    uint16_t* hbuf;              // [T*k, I] bf16, grouped position order
     float* obuf;                 // [T*k, H] fp32, entry order t*k+j
     int* err;
 };
-
-__device__ __forceinline__ void mma_bf16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void fill_lut(Fp4Lut* lut) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = make_fp4_lut(static_cast<uint32_t>(i));
-}
-
-__device__ __forceinline__ uint32_t word(const uint4& v, int j) {
-    return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
-}
 
 // -------------------------------------------------------------------- combine
 // y[t] = sum_j w[t, j] * o[t*k + j] in fixed j order; optional residual

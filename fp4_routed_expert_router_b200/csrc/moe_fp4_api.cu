@@ -15,8 +15,7 @@
 #include "../../include/moe_fp4.h"
 #include "common.cuh"
 #include "decode_common.cuh"
-#include "decode_tile.cuh"
-#include "fp4_decode.cuh"
+#include "decode_fused.cuh"
 #include "router.cuh"
 #include "slot_layout.cuh"
 #include "residency.h"
@@ -33,13 +32,20 @@ struct moe_fp4_ctx {
     uint8_t* arena = nullptr;
     bool own_arena = false;
     int32_t* d_table = nullptr;        // [L][E]
+    uint8_t* d_rowref = nullptr;       // [n_slots][2I + H] largest scale byte of each weight row
     uint8_t* d_staging = nullptr;      // one expert, checkpoint layout
-    uint16_t* d_h = nullptr;           // [max_tokens*k, I] bf16
+    uint16_t* d_xh = nullptr;          // [max_tokens*k, H] f16 prescaled x rows (decode kernel)
+    float* d_xs = nullptr;             // [max_tokens*k] their 2^-sigma
+    uint16_t* d_hh = nullptr;          // [max_tokens*k, I] f16 prescaled h rows
+    float* d_hs = nullptr;             // [max_tokens*k, I/32] 2^-sigma per (entry, 32-K block)
     float* d_o = nullptr;              // [max_tokens*k, H] fp32
     float* d_norm = nullptr;           // [max_tokens*k] fp32 (saliency)
     int32_t* d_grp = nullptr;          // expert_outputs grouping: counts [E], offsets [E+1], perm [max_tokens*k]
+    int* d_tile = nullptr;             // [H/32] combine counters of the decode kernel
+    unsigned int* d_gbar = nullptr;    // [4] grid barriers of the decode kernel
     int* d_err = nullptr;              // error word [4]
     unsigned int* d_ticket = nullptr;  // route kernel ticket
+    unsigned long long timeout_ns = 1000000000ull;   // bounded device waits
     std::vector<int32_t> h_table;      // host mirror of d_table
     std::vector<int64_t> slot_owner;   // slot -> layer*E+expert or -1
     int path = MOE_FP4_PATH_AUTO;
@@ -139,70 +145,57 @@ cudaError_t launch_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim
 
 // Re-lay one expert from the staging buffer (checkpoint layout: w1, w3, w2
 // codes, then s1, s3, s2 scales, row-major) into its slot (slot_layout.cuh):
-// one thread per 16-byte chunk of codes (re-encoded, placed in its block at
-// its swizzled position) and one thread per scale byte (checked against the
-// supported range [2, 252]).  Thread 0 maps (layer, expert) -> slot.
+// one thread per 16-byte chunk of codes (four words gathered from the row's
+// 64-byte group, placed in its block at its swizzled position), one per scale
+// byte (checked against the supported range [2, 252]), and one per weight row
+// for the row's largest scale byte (rowref, used by the tcgen05 path).
+// Thread 0 maps (layer, expert) -> slot.
 __global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, SlotLayout L,
-                                 int32_t* table, int map_index, int slot, int* err) {
-    const size_t H = L.H, I = L.I, KBu = L.KBu, nfu = L.nfu, KBd = L.KBd, nfd = L.nfd;
+                                 uint8_t* __restrict__ rowref, int32_t* table, int map_index, int slot, int* err) {
+    const size_t H = L.H, I = L.I;
     const size_t n13 = I * H / 32, n2 = H * I / 32;        // 16-byte code chunks of w1 (w3), w2
     const size_t s13 = I * H / 32, s2 = H * I / 32;        // scale bytes of s1 (s3), s2
+    const size_t sbase = 3 * I * H / 2;                      // scales start after the codes
     const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
     if (i == 0 && map_index >= 0) table[map_index] = slot;
     if (i < 2 * n13 + n2) {
         size_t so, dofs;
-        if (i < 2 * n13) {                                   // w1 / w3 chunk
-            const size_t mat = i / n13, rem = i - mat * n13;
-            const size_t r = rem / (H / 32), q = rem - r * (H / 32);
-            const size_t f = q / (KBu / 32), qi = q - f * (KBu / 32);
-            so = mat * (I * H / 2) + r * (H / 2) + q * 16;
-            dofs = ((r / 16) * nfu + f) * L.UB + mat * 16 * (KBu / 2) + (r % 16) * (KBu / 2) +
-                   static_cast<size_t>(swizzle_chunk(static_cast<int>(qi), static_cast<int>(r % 16),
-                                                     static_cast<int>(KBu / 2))) * 16;
-        } else {                                             // w2 chunk
-            const size_t rem = i - 2 * n13;
-            const size_t r = rem / (I / 32), q = rem - r * (I / 32);
-            const size_t f = q / (KBd / 32), qi = q - f * (KBd / 32);
-            so = I * H + r * (I / 2) + q * 16;
-            dofs = L.up_bytes + ((r / 16) * nfd + f) * L.DB + (r % 16) * (KBd / 2) +
-                   static_cast<size_t>(swizzle_chunk(static_cast<int>(qi), static_cast<int>(r % 16),
-                                                     static_cast<int>(KBd / 2))) * 16;
-        }
-        const uint4 v = *reinterpret_cast<const uint4*>(src + so);
+        slot_code_chunk(L, i, &so, &dofs);
         uint4 w;
-        w.x = fp4_reencode_word(v.x);
-        w.y = fp4_reencode_word(v.y);
-        w.z = fp4_reencode_word(v.z);
-        w.w = fp4_reencode_word(v.w);
+        w.x = *reinterpret_cast<const uint32_t*>(src + so + 0);
+        w.y = *reinterpret_cast<const uint32_t*>(src + so + 16);
+        w.z = *reinterpret_cast<const uint32_t*>(src + so + 32);
+        w.w = *reinterpret_cast<const uint32_t*>(src + so + 48);
         *reinterpret_cast<uint4*>(dst + dofs) = w;
         return;
     }
     const size_t b = i - (2 * n13 + n2);
-    if (b >= 2 * s13 + s2) return;
-    const size_t sbase = 3 * I * H / 2;                      // scales start after the codes
-    size_t dofs;
-    if (b < 2 * s13) {                                       // s1 / s3 byte
-        const size_t mat = b / s13, rem = b - mat * s13;
-        const size_t r = rem / (H / 32), q = rem - r * (H / 32);
-        const size_t f = q / (KBu / 32), qi = q - f * (KBu / 32);
-        dofs = ((r / 16) * nfu + f) * L.UB + 32 * (KBu / 2) + mat * 16 * (KBu / 32) + (r % 16) * (KBu / 32) + qi;
-    } else {                                                 // s2 byte
-        const size_t rem = b - 2 * s13;
-        const size_t r = rem / (I / 32), q = rem - r * (I / 32);
-        const size_t f = q / (KBd / 32), qi = q - f * (KBd / 32);
-        dofs = L.up_bytes + ((r / 16) * nfd + f) * L.DB + 16 * (KBd / 2) + (r % 16) * (KBd / 32) + qi;
+    if (b < 2 * s13 + s2) {
+        const uint8_t v = src[sbase + b];
+        dst[slot_scale_byte(L, b)] = v;
+        if (v < 2 || v > 252) latch_error(err, ERR_EINVAL, static_cast<int>(b), KID_LOAD);
+        return;
     }
-    const uint8_t v = src[sbase + b];
-    dst[dofs] = v;
-    if (v < 2 || v > 252) latch_error(err, ERR_EINVAL, static_cast<int>(b), KID_LOAD);
+    const size_t r = b - (2 * s13 + s2);                     // weight row: w1 rows, w3 rows, w2 rows
+    if (r >= 2 * I + H || rowref == nullptr) return;
+    const size_t n = r < 2 * I ? H / 32 : I / 32;
+    const uint8_t* sp = src + sbase + (r < 2 * I ? r * (H / 32) : 2 * s13 + (r - 2 * I) * (I / 32));
+    uint8_t mx = 0;
+    for (size_t j = 0; j < n; ++j) mx = sp[j] > mx ? sp[j] : mx;
+    rowref[static_cast<size_t>(slot) * (2 * I + H) + r] = mx;
+}
+
+inline size_t load_threads(const SlotLayout& L) {
+    const size_t H = L.H, I = L.I;
+    return 3 * I * H / 32 + 3 * I * H / 32 + 2 * I + H;   // code chunks + scale bytes + rows
 }
 
 const char* kernel_name(int kid) {
     switch (kid) {
         case KID_ROUTE: return "route";
         case KID_LOAD: return "load_expert_slot";
-        case KID_UP: return "gemv_up";
-        case KID_DOWN: return "gemv_down";
+        case KID_UP: return "decode_layer (w1/w3)";
+        case KID_DOWN: return "decode_layer (w2)";
         case KID_COMBINE: return "combine";
         case KID_TC_UP: return "tc_up";
         case KID_TC_DOWN: return "tc_down";
@@ -211,68 +204,115 @@ const char* kernel_name(int kid) {
     }
 }
 
-// ---- decode path: the tile-streaming GEMV kernels (decode_tile.cuh)
-// Instantiated shapes (RB, KS, CPW):
-//   up   RB 1: 40 chunks (H 5120) -> KS 10 x CPW 4; 2 chunks (H 256) -> 2 x 1
-//   down RB 2: 18 chunks (I 2304) -> KS  9 x CPW 2; 1 chunk  (I 128) -> 1 x 1
-template <bool UP, int RB, int KS, int CPW>
-cudaError_t launch_tile(moe_fp4_ctx* c, dim3 grid, cudaStream_t s, const GemvArgs& a, const SlotLayout& L,
-                        const TilePlan& p) {
-    const dim3 block((RB * KS + 1) * 32);
-    if (c) return launch_k(c, UP ? "gemv_up" : "gemv_down", gemv_tile_kernel<UP, RB, KS, CPW>, grid, block,
-                           static_cast<size_t>(p.smem_bytes), s, a, L, p);
-    return launch_pdl(gemv_tile_kernel<UP, RB, KS, CPW>, grid, block, static_cast<size_t>(p.smem_bytes), s, a, L, p);
+// ---- decode path: the persistent fused layer kernel (decode_fused.cuh)
+// Instantiated for NTOK in {1, 8} (a batch of one token keeps one partial
+// column) and K blocks of 128 or 256 for w1/w3 (QU) and w2 (QD).
+template <int NTOK, int QU, int QD>
+cudaError_t launch_decode_t(const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid,
+                            cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(p.smem_bytes);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs co-resident: the kernel has grid barriers
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, moe_fp4_decode_layer<NTOK, QU, QD>, a, L, p);
 }
 
-template <bool UP, int RB, int KS, int CPW>
-cudaError_t allow_tile_smem(int bytes) {
-    return cudaFuncSetAttribute(reinterpret_cast<const void*>(gemv_tile_kernel<UP, RB, KS, CPW>),
+template <int NTOK, int QU, int QD>
+cudaError_t allow_decode_smem(int bytes) {
+    return cudaFuncSetAttribute(reinterpret_cast<const void*>(moe_fp4_decode_layer<NTOK, QU, QD>),
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
-bool decode_shape_ok(const SlotLayout& L) {
-    const int cu = L.H / 128, cd = L.I / 128;
-    return (cu == 40 || cu == 2) && (cd == 18 || cd == 1) && L.H % 32 == 0;
 }
 
 cudaError_t allow_decode_smem_all(int bytes) {
     cudaError_t e = cudaSuccess, r;
-    if ((r = allow_tile_smem<true, 1, 8, 5>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_tile_smem<true, 1, 2, 1>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_tile_smem<false, 2, 6, 3>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_tile_smem<false, 2, 1, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<1, 1, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<1, 1, 2>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<1, 2, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<1, 2, 2>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<8, 1, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<8, 1, 2>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<8, 2, 1>(bytes)) != cudaSuccess) e = r;
+    if ((r = allow_decode_smem<8, 2, 2>(bytes)) != cudaSuccess) e = r;
     return e;
 }
 
-// Launch up then down (c may be NULL: no profiling).  smem_limit: opt-in
-// shared memory per block minus the kernels' static shared memory.
-cudaError_t decode_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& L, int active_max, int sm_count,
-                           int smem_limit, cudaStream_t s) {
-    if (!decode_shape_ok(L)) return cudaErrorNotSupported;
-    const bool big_up = (L.H / 128 == 40), big_down = (L.I / 128 == 18);
-    const TilePlan pu = make_tile_plan(true, L, 1, big_up ? 8 : 2, a.E, active_max, smem_limit);
-    const TilePlan pd = make_tile_plan(false, L, 2, big_down ? 12 : 2, a.E, active_max, smem_limit);
-    if (!pu.stages || !pd.stages) return cudaErrorNotSupported;
-    const dim3 grid(static_cast<unsigned>(sm_count));
-    cudaError_t e = big_up ? launch_tile<true, 1, 8, 5>(c, grid, s, a, L, pu)
-                           : launch_tile<true, 1, 2, 1>(c, grid, s, a, L, pu);
-    if (e != cudaSuccess) return e;
-    return big_down ? launch_tile<false, 2, 6, 3>(c, grid, s, a, L, pd)
-                    : launch_tile<false, 2, 1, 1>(c, grid, s, a, L, pd);
+cudaError_t launch_decode(const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid, cudaStream_t s) {
+    const bool qu = L.KBu == 256, qd = L.KBd == 256;
+    if (p.tp == 1) {
+        if (qu) return qd ? launch_decode_t<1, 2, 2>(a, L, p, grid, s) : launch_decode_t<1, 2, 1>(a, L, p, grid, s);
+        return qd ? launch_decode_t<1, 1, 2>(a, L, p, grid, s) : launch_decode_t<1, 1, 1>(a, L, p, grid, s);
+    }
+    if (qu) return qd ? launch_decode_t<8, 2, 2>(a, L, p, grid, s) : launch_decode_t<8, 2, 1>(a, L, p, grid, s);
+    return qd ? launch_decode_t<8, 1, 2>(a, L, p, grid, s) : launch_decode_t<8, 1, 1>(a, L, p, grid, s);
 }
 
-// tcgen05 path: gather x rows by expert, then the up and down GEMMs.
-cudaError_t tc_forward(moe_fp4_ctx* c, const GemvArgs& a, const SlotLayout& L, int T, cudaStream_t s) {
+// Launch the decode kernel bracketed by profiling events when the context
+// profiles (c may be NULL).
+cudaError_t decode_run(moe_fp4_ctx* c, const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid,
+                       cudaStream_t s) {
+    const bool prof = c && c->profile && c->prof.size() < 65536;
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    if (prof) {
+        ea = take_event(c);
+        eb = take_event(c);
+        cudaEventRecord(ea, s);
+    }
+    cudaError_t e = launch_decode(a, L, p, grid, s);
+    if (prof) {
+        cudaEventRecord(eb, s);
+        c->prof.push_back({"decode_layer", ea, eb});
+    }
+    return e;
+}
+
+// Decode arguments over the context's workspace.
+DecodeArgs decode_args(moe_fp4_ctx* c, int layer, int k, int T, const uint16_t* x) {
+    DecodeArgs a{};
+    a.arena = c->arena;
+    a.slot_bytes = c->slot_bytes;
+    a.slot_table = c->d_table;
+    a.layer = layer;
+    a.E = c->cfg.n_experts;
+    a.k = k;
+    a.H = c->cfg.hidden;
+    a.I = c->cfg.inter;
+    a.T = T;
+    a.x = x;
+    a.xh = c->d_xh;
+    a.xs = c->d_xs;
+    a.hh = c->d_hh;
+    a.hs = c->d_hs;
+    a.obuf = c->d_o;
+    a.tile_cnt = c->d_tile;
+    a.gbar = c->d_gbar;
+    a.err = c->d_err;
+    a.timeout_ns = c->timeout_ns;
+    return a;
+}
+
+// tcgen05 path: gather x rows by expert (prescaled f16), up GEMM (bf16 h),
+// h -> prescaled f16, down GEMM.
+cudaError_t tc_forward(moe_fp4_ctx* c, const ExpertArgs& a, const SlotLayout& L, int T, cudaStream_t s) {
     const TcPlan& p = c->tc;
     if (!p.ready) return cudaErrorNotSupported;
     const int rows = T * a.k;
     cudaError_t e = launch_k(c, "gather", gather_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, s,
-                             a.x, a.perm, a.k, a.H, rows, p.xg);
+                             a.x, a.perm, a.k, a.H, rows, p.xg, p.xcs);
     if (e != cudaSuccess) return e;
-    const TcArgs tu = tc_args(p, a, L, T, true), td = tc_args(p, a, L, T, false);
+    TcArgs tu = tc_args(p, a, L, T, true, c->d_rowref), td = tc_args(p, a, L, T, false, c->d_rowref);
     if (!tu.centries || !td.centries) return cudaErrorNotSupported;
+    tu.timeout_ns = td.timeout_ns = c->timeout_ns;
     const dim3 grid(static_cast<unsigned>(p.sm_count)), block(kTcThreads);
     e = launch_k(c, "tc_up", tc_gemm_kernel<true>, grid, block, tc_smem_bytes(tu), s, tu, p.map_x);
+    if (e != cudaSuccess) return e;
+    e = launch_k(c, "h_convert", h_convert_kernel, dim3(static_cast<unsigned>((rows * 32 + 255) / 256)), dim3(256), 0,
+                 s, static_cast<const uint16_t*>(p.hb), a.I, rows, p.hh, p.hcs);
     if (e != cudaSuccess) return e;
     return launch_k(c, "tc_down", tc_gemm_kernel<false>, grid, block, tc_smem_bytes(td), s, td, p.map_h);
 }
@@ -318,12 +358,19 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         c->own_arena = true;
     }
     const size_t ent = static_cast<size_t>(cfg->max_tokens) * cfg->top_k;
+    const size_t rowref_bytes = static_cast<size_t>(cfg->n_slots) * (2 * I + H);
     if (cudaMalloc(&c->d_table, sizeof(int32_t) * L * E) != cudaSuccess ||
+        cudaMalloc(&c->d_rowref, rowref_bytes) != cudaSuccess ||
         cudaMalloc(&c->d_staging, c->slot_bytes) != cudaSuccess ||
-        cudaMalloc(&c->d_h, sizeof(uint16_t) * ent * I) != cudaSuccess ||
+        cudaMalloc(&c->d_xh, sizeof(uint16_t) * ent * H) != cudaSuccess ||
+        cudaMalloc(&c->d_xs, sizeof(float) * ent) != cudaSuccess ||
+        cudaMalloc(&c->d_hh, sizeof(uint16_t) * ent * I) != cudaSuccess ||
+        cudaMalloc(&c->d_hs, sizeof(float) * ent * (I / 32)) != cudaSuccess ||
         cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
         cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
         cudaMalloc(&c->d_grp, sizeof(int32_t) * (2 * static_cast<size_t>(cfg->n_experts) + 1 + ent)) != cudaSuccess ||
+        cudaMalloc(&c->d_tile, sizeof(int) * (H / 32)) != cudaSuccess ||
+        cudaMalloc(&c->d_gbar, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
         cudaGetLastError();
@@ -334,11 +381,14 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaGetLastError();
         return bail(MOE_FP4_ECUDA);
     }
-    if (tc_plan_create(&c->tc, *cfg, c->d_h, c->sm_count, c->smem_optin) != cudaSuccess) {
+    if (tc_plan_create(&c->tc, *cfg, c->d_hh, c->sm_count, c->smem_optin) != cudaSuccess) {
         cudaGetLastError();
         return bail(MOE_FP4_ENOMEM);
     }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
+        cudaMemset(c->d_rowref, 0, rowref_bytes) != cudaSuccess ||
+        cudaMemset(c->d_tile, 0, sizeof(int) * (H / 32)) != cudaSuccess ||
+        cudaMemset(c->d_gbar, 0, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
         cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
@@ -355,11 +405,17 @@ void moe_fp4_destroy(moe_fp4_ctx* c) {
     cudaDeviceSynchronize();
     if (c->own_arena) cudaFree(c->arena);
     cudaFree(c->d_table);
+    cudaFree(c->d_rowref);
     cudaFree(c->d_staging);
-    cudaFree(c->d_h);
+    cudaFree(c->d_xh);
+    cudaFree(c->d_xs);
+    cudaFree(c->d_hh);
+    cudaFree(c->d_hs);
     cudaFree(c->d_o);
     cudaFree(c->d_norm);
     cudaFree(c->d_grp);
+    cudaFree(c->d_tile);
+    cudaFree(c->d_gbar);
     for (int b = 0; b < 2; ++b) {
         if (c->d_stage2[b]) cudaFree(c->d_stage2[b]);
         if (c->st_ready[b]) cudaEventDestroy(c->st_ready[b]);
@@ -384,6 +440,10 @@ moe_fp4_status moe_fp4_set_option(moe_fp4_ctx* c, int option, int value) {
     }
     if (option == MOE_FP4_OPT_PROFILE && (value == 0 || value == 1)) {
         c->profile = value != 0;
+        return MOE_FP4_OK;
+    }
+    if (option == MOE_FP4_OPT_WAIT_LIMIT_US && value >= 0 && value <= 10000000) {
+        c->timeout_ns = value == 0 ? 1000000000ull : static_cast<unsigned long long>(value) * 1000ull;
         return MOE_FP4_OK;
     }
     return host_fail(c, MOE_FP4_EINVAL, "set_option: unknown option %d / value %d", option, value);
@@ -427,10 +487,10 @@ moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx* c, int layer, int expert, i
         e = cudaMemcpyAsync(c->d_staging + p.off, p.p, p.n, cudaMemcpyDefault, s);
         if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: copy");
     }
-    const size_t threads = 3 * I * H / 32 + 3 * I * H / 32;  // code chunks + scale bytes
+    const size_t threads = load_threads(c->lay);
     load_slot_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-        c->d_staging, c->arena + static_cast<size_t>(slot) * c->slot_bytes, c->lay, c->d_table, idx, slot,
-        c->d_err);
+        c->d_staging, c->arena + static_cast<size_t>(slot) * c->slot_bytes, c->lay, c->d_rowref, c->d_table, idx,
+        slot, c->d_err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(c, e, "load_expert_slot: launch");
     c->h_table[idx] = slot;
@@ -479,7 +539,7 @@ moe_fp4_status moe_fp4_stream_experts(moe_fp4_ctx* c, int layer, const int32_t* 
                   keys.data(), n, slot.data(), hit.data(), evicted.data()))
         return host_fail(c, MOE_FP4_EINVAL, "stream_experts: no slot plan");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t threads = 3 * static_cast<size_t>(g.inter) * g.hidden / 16;   // code chunks + scale bytes
+    const size_t threads = load_threads(c->lay);
     for (int i = 0; i < n; ++i) {
         if (hit[i]) {
             ++c->stream_stats[0];
@@ -497,8 +557,8 @@ moe_fp4_status moe_fp4_stream_experts(moe_fp4_ctx* c, int layer, const int32_t* 
             (e = cudaMemsetAsync(c->d_table + evicted[i], 0xFF, sizeof(int32_t), s)) != cudaSuccess)
             return cuda_fail(c, e, "stream_experts: evict");
         load_slot_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-            c->d_stage2[b], c->arena + static_cast<size_t>(slot[i]) * c->slot_bytes, c->lay, c->d_table,
-            static_cast<int>(keys[i]), slot[i], c->d_err);
+            c->d_stage2[b], c->arena + static_cast<size_t>(slot[i]) * c->slot_bytes, c->lay, c->d_rowref,
+            c->d_table, static_cast<int>(keys[i]), slot[i], c->d_err);
         if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaEventRecord(c->st_free[b], s)) != cudaSuccess)
             return cuda_fail(c, e, "stream_experts: relayout");
         ++c->stream_stats[1];
@@ -563,18 +623,73 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     (void)counts;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int H = g.hidden, I = g.inter, E = g.n_experts, k = g.top_k;
-    const int ent = T * k;
-    const int active_max = ent < E ? ent : E;
-    GemvArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_h, c->d_o, c->d_err};
-    const bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
-    cudaError_t e = use_tc ? tc_forward(c, a, c->lay, T, s)
-                           : decode_forward(c, a, c->lay, active_max, c->sm_count, c->smem_optin, s);
+    const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
+    if (!want_tc) {   // decode path: one persistent kernel (+ the combine for batches above 16 tokens)
+        const DecodePlan p = make_decode_plan(c->lay, T, k, E, false, c->smem_optin, c->sm_count);
+        if (p.ok) {
+            DecodeArgs a = decode_args(c, layer, k, T, x);
+            a.weights = const_cast<float*>(weights);
+            a.offsets = const_cast<int32_t*>(offsets);
+            a.perm = const_cast<int32_t*>(perm);
+            const bool fuse = T <= kDecCombineMax;
+            a.y = fuse ? y : nullptr;
+            a.x_out = fuse ? x_out : nullptr;
+            cudaError_t e = decode_run(c, a, c->lay, p, c->sm_count, s);
+            if (e != cudaSuccess) return cuda_fail(c, e, "forward: decode launch");
+            if (fuse) return MOE_FP4_OK;
+            const int n4 = T * (H / 4);
+            e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
+                         static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
+            return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "forward: combine launch");
+        }
+        if (c->path == MOE_FP4_PATH_GEMV)
+            return host_fail(c, MOE_FP4_EINVAL, "forward: T %d does not fit the decode kernel", T);
+    }
+    ExpertArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, k, H, I, x, offsets, perm, c->d_o, c->d_err};
+    cudaError_t e = tc_forward(c, a, c->lay, T, s);
     if (e != cudaSuccess) return cuda_fail(c, e, "forward: expert FFN launch");
     const int n4 = T * (H / 4);
     e = launch_k(c, "combine", combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s,
                  static_cast<const float*>(c->d_o), weights, x, T, H, k, y, x_out);
     if (e != cudaSuccess) return cuda_fail(c, e, "forward: combine launch");
     return MOE_FP4_OK;
+}
+
+moe_fp4_status moe_fp4_route_forward(moe_fp4_ctx* c, int layer, const float* logits, const uint8_t* keep_mask,
+                                     const uint16_t* x, int T, int32_t* ids, float* weights, int32_t* counts,
+                                     int32_t* offsets, int32_t* perm, float* y, uint16_t* x_out, void* stream) {
+    if (!c) return MOE_FP4_EINVAL;
+    const moe_fp4_config& g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers || T < 0 || T > g.max_tokens)
+        return host_fail(c, MOE_FP4_EINVAL, "route_forward: layer %d / T %d out of range", layer, T);
+    if (!counts || !offsets) return host_fail(c, MOE_FP4_EINVAL, "route_forward: NULL output");
+    if (T > 0 && (!logits || !x || !ids || !weights || !perm || !y))
+        return host_fail(c, MOE_FP4_EINVAL, "route_forward: NULL argument");
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
+        (reinterpret_cast<uintptr_t>(x_out) & 7) || (reinterpret_cast<uintptr_t>(weights) & 3))
+        return host_fail(c, MOE_FP4_EINVAL, "route_forward: x and y must be 16-byte aligned, x_out 8-byte");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
+    if (T > 0 && !want_tc) {
+        const DecodePlan p = make_decode_plan(c->lay, T, g.top_k, g.n_experts, true, c->smem_optin, c->sm_count);
+        if (p.ok) {   // routing inside the layer kernel: one launch for the whole layer
+            DecodeArgs a = decode_args(c, layer, g.top_k, T, x);
+            a.logits = logits;
+            a.keep = keep_mask;
+            a.ids = ids;
+            a.weights = weights;
+            a.counts = counts;
+            a.offsets = offsets;
+            a.perm = perm;
+            a.y = y;
+            a.x_out = x_out;
+            cudaError_t e = decode_run(c, a, c->lay, p, c->sm_count, s);
+            return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "route_forward: decode launch");
+        }
+    }
+    moe_fp4_status st = moe_fp4_route(c, layer, logits, keep_mask, T, ids, weights, counts, offsets, perm, stream);
+    if (st != MOE_FP4_OK || T == 0) return st;
+    return moe_fp4_forward(c, layer, x, T, ids, weights, counts, offsets, perm, y, x_out, stream);
 }
 
 moe_fp4_status moe_fp4_expert_outputs(moe_fp4_ctx* c, int layer, const uint16_t* x, int n, const int32_t* experts,
@@ -598,10 +713,22 @@ moe_fp4_status moe_fp4_expert_outputs(moe_fp4_ctx* c, int layer, const uint16_t*
     cudaError_t e = launch_k(c, "group", group_kernel, dim3(1), dim3(kRouteWarps * 32),
                              sizeof(int) * kRouteWarps * E, s, ra);
     if (e != cudaSuccess) return cuda_fail(c, e, "expert_outputs: group launch");
-    GemvArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, 1, H, I, x, offsets, perm, c->d_h, o, c->d_err};
-    const bool use_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && 4LL * n >= 3LL * E);
-    e = use_tc ? tc_forward(c, a, c->lay, n, s)
-               : decode_forward(c, a, c->lay, n < E ? n : E, c->sm_count, c->smem_optin, s);
+    const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && 4LL * n >= 3LL * E);
+    if (!want_tc) {
+        const DecodePlan p = make_decode_plan(c->lay, n, 1, E, false, c->smem_optin, c->sm_count);
+        if (p.ok) {   // every row its own token (k = 1), per-entry outputs only
+            DecodeArgs a = decode_args(c, layer, 1, n, x);
+            a.offsets = offsets;
+            a.perm = perm;
+            a.obuf = o;
+            e = decode_run(c, a, c->lay, p, c->sm_count, s);
+            return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "expert_outputs: decode launch");
+        }
+        if (c->path == MOE_FP4_PATH_GEMV)
+            return host_fail(c, MOE_FP4_EINVAL, "expert_outputs: n %d does not fit the decode kernel", n);
+    }
+    ExpertArgs a{c->arena, c->slot_bytes, c->d_table, layer, E, 1, H, I, x, offsets, perm, o, c->d_err};
+    e = tc_forward(c, a, c->lay, n, s);
     if (e != cudaSuccess) return cuda_fail(c, e, "expert_outputs: expert FFN launch");
     return MOE_FP4_OK;
 }
@@ -696,8 +823,8 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx* c, char* msg, size_t n) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
-// Forward without allocation (moe_fp4_forward_noalloc): the decode kernels
-// with their scratch in a file-scope device array instead of a context
+// Forward without allocation (moe_fp4_forward_noalloc): the decode kernel
+// with its scratch in a file-scope device array instead of a context
 // workspace.  Host code must not use the array's name as a device address:
 // its device address is looked up once per device with cudaGetSymbolAddress.
 namespace {
@@ -705,18 +832,21 @@ namespace {
 constexpr size_t kNoallocScratchBytes = size_t(16) << 20;   // 16 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 __device__ int g_noalloc_err_sink[4];                        // errors when err == NULL
+// Grid-barrier state of the decode kernel: it must start at zero and every
+// launch leaves it at zero again.
+__device__ unsigned int g_noalloc_gbar[4] = {0u, 0u, 0u, 0u};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 
-// Device addresses of the scratch array and the error sink on the current
-// device (looked up on the first call per device).
 // Per-device set-up on the first call (that device current): the device
-// addresses of the scratch array and of the error sink, the SM count, the
-// opt-in shared memory, and the kernels' shared-memory attribute.
+// addresses of the scratch array, the error sink and the barrier state, the
+// SM count, the opt-in shared memory, and the kernels' shared-memory
+// attribute.
 struct NoallocDevice {
     void* scratch;
     int* sink;
+    unsigned int* gbar;
     int sm_count;
     int smem_limit;
 };
@@ -729,14 +859,17 @@ bool noalloc_setup(int dev, NoallocDevice* out) {
     if (!d.scratch) {
         void* p = nullptr;
         void* q = nullptr;
+        void* gb = nullptr;
         int sms = 0, optin = 0;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return false;
         if (cudaGetSymbolAddress(&q, g_noalloc_err_sink) != cudaSuccess) return false;
+        if (cudaGetSymbolAddress(&gb, g_noalloc_gbar) != cudaSuccess) return false;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
         optin -= 1024;
         if (allow_decode_smem_all(optin) != cudaSuccess) return false;
         d.sink = static_cast<int*>(q);
+        d.gbar = static_cast<unsigned int*>(gb);
         d.sm_count = sms;
         d.smem_limit = optin;
         d.scratch = p;
@@ -744,6 +877,8 @@ bool noalloc_setup(int dev, NoallocDevice* out) {
     *out = d;
     return true;
 }
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 }  // namespace
 
@@ -757,30 +892,58 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
     if (T == 0) return MOE_FP4_OK;
     if (!x || !weights || !offsets || !perm || !y) return MOE_FP4_EINVAL;
     if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(y) & 15) ||
-        (reinterpret_cast<uintptr_t>(x_out) & 7) || (reinterpret_cast<uintptr_t>(arena) & 255))
+        (reinterpret_cast<uintptr_t>(x_out) & 7) || (reinterpret_cast<uintptr_t>(weights) & 3) ||
+        (reinterpret_cast<uintptr_t>(arena) & 255))
         return MOE_FP4_EINVAL;
     const size_t H = cfg->hidden, I = cfg->inter, k = cfg->top_k, E = cfg->n_experts;
     const size_t ent = static_cast<size_t>(T) * k;
-    const size_t h_bytes = (ent * I * sizeof(uint16_t) + 255) & ~size_t(255);
-    const size_t need = h_bytes + ent * H * sizeof(float);
+    // scratch: x rows (f16) and their scales, h rows (f16) and block scales,
+    // per-entry outputs, combine counters
+    const size_t o_xh = 0, o_xs = align256(o_xh + T * H * 2), o_hh = align256(o_xs + T * 4);
+    const size_t o_hs = align256(o_hh + ent * I * 2), o_o = align256(o_hs + ent * (I / 32) * 4);
+    const size_t o_tc = align256(o_o + ent * H * 4), need = o_tc + (H / 32) * 4;
     if (need > kNoallocScratchBytes) return MOE_FP4_EINVAL;
+    const SlotLayout L = make_slot_layout(cfg->hidden, cfg->inter);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_FP4_ECUDA;
     NoallocDevice d{};
     if (!noalloc_setup(dev, &d)) return MOE_FP4_ECUDA;
+    const DecodePlan p = make_decode_plan(L, T, static_cast<int>(k), static_cast<int>(E), false, d.smem_limit, d.sm_count);
+    if (!p.ok) return MOE_FP4_EINVAL;                         // shape or batch the decode kernel does not take
     uint8_t* sp = static_cast<uint8_t*>(d.scratch);
-    GemvArgs a{arena, moe_fp4_slot_bytes(cfg), slot_table, layer, static_cast<int>(E), static_cast<int>(k),
-               static_cast<int>(H), static_cast<int>(I), x, offsets, perm,
-               reinterpret_cast<uint16_t*>(sp), reinterpret_cast<float*>(sp + h_bytes),
-               err ? reinterpret_cast<int*>(err) : d.sink};
+    DecodeArgs a{};
+    a.arena = arena;
+    a.slot_bytes = moe_fp4_slot_bytes(cfg);
+    a.slot_table = slot_table;
+    a.layer = layer;
+    a.E = static_cast<int>(E);
+    a.k = static_cast<int>(k);
+    a.H = static_cast<int>(H);
+    a.I = static_cast<int>(I);
+    a.T = T;
+    a.weights = const_cast<float*>(weights);
+    a.offsets = const_cast<int32_t*>(offsets);
+    a.perm = const_cast<int32_t*>(perm);
+    a.x = x;
+    a.xh = reinterpret_cast<uint16_t*>(sp + o_xh);
+    a.xs = reinterpret_cast<float*>(sp + o_xs);
+    a.hh = reinterpret_cast<uint16_t*>(sp + o_hh);
+    a.hs = reinterpret_cast<float*>(sp + o_hs);
+    a.obuf = reinterpret_cast<float*>(sp + o_o);
+    a.tile_cnt = reinterpret_cast<int*>(sp + o_tc);
+    a.gbar = d.gbar;
+    const bool fuse = T <= kDecCombineMax;                    // else the combine kernel follows
+    a.y = fuse ? y : nullptr;
+    a.x_out = fuse ? x_out : nullptr;
+    a.err = err ? reinterpret_cast<int*>(err) : d.sink;
+    a.timeout_ns = 1000000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int active_max = static_cast<int>(ent < E ? ent : E);
-    if (decode_forward(nullptr, a, make_slot_layout(cfg->hidden, cfg->inter), active_max, d.sm_count, d.smem_limit,
-                     s) != cudaSuccess)
-        return MOE_FP4_ECUDA;
-    const int n4 = T * static_cast<int>(H / 4);
-    if (launch_pdl(combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s, static_cast<const float*>(a.obuf),
-                   weights, x, T, static_cast<int>(H), static_cast<int>(k), y, x_out) != cudaSuccess)
-        return MOE_FP4_ECUDA;
+    if (launch_decode(a, L, p, d.sm_count, s) != cudaSuccess) return MOE_FP4_ECUDA;
+    if (!fuse) {
+        const int n4 = T * static_cast<int>(H / 4);
+        if (launch_pdl(combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s, static_cast<const float*>(a.obuf),
+                       weights, x, T, static_cast<int>(H), static_cast<int>(k), y, x_out) != cudaSuccess)
+            return MOE_FP4_ECUDA;
+    }
     return MOE_FP4_OK;
 }

@@ -46,30 +46,33 @@ struct RouteArgs {
     int* err;
 };
 
+// Top-k of one token's logits by one warp: writes the k chosen experts (in
+// the total order) to ids_out[0..k) and their renormalised weights to
+// w_out[0..k).  NaN logits, or fewer than k selectable experts, latch EINVAL.
 template <int NI>   // logits held per lane: E <= 32 * NI
-__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane) {
-    const float* l = a.logits + static_cast<size_t>(t) * a.E;
+__device__ __forceinline__ void route_one(const float* l, const uint8_t* keep, int E, int k, int t, int lane,
+                                          int32_t* ids_out, float* w_out, int* err) {
     uint32_t key[NI];
     bool nan = false;
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
         int e = lane + 32 * i;
         key[i] = 0;
-        if (e < a.E) {
+        if (e < E) {
             float v = __ldg(l + e);
             nan |= (v != v);
-            bool ok = (a.keep == nullptr) || (__ldg(a.keep + e) != 0);
+            bool ok = (keep == nullptr) || (__ldg(keep + e) != 0);
             key[i] = ok ? orderable(v) : 0u;
         }
     }
     if (__any_sync(0xFFFFFFFFu, nan)) {
-        if (lane == 0) latch_error(a.err, ERR_EINVAL, t, KID_ROUTE);
+        if (lane == 0) latch_error(err, ERR_EINVAL, t, KID_ROUTE);
     }
     uint32_t removed = 0;
     int my_id = 0;
     float my_val = 0.f;
     bool short_of_experts = false;
-    for (int r = 0; r < a.k; ++r) {
+    for (int r = 0; r < k; ++r) {
         uint32_t best = 0;
         int bi = 0;
 #pragma unroll
@@ -85,17 +88,23 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane)
         if (lane == r) { my_id = static_cast<int>(win); my_val = from_orderable(wmax); }
     }
     if (short_of_experts) {
-        if (lane == 0) latch_error(a.err, ERR_EINVAL, t, KID_ROUTE);
+        if (lane == 0) latch_error(err, ERR_EINVAL, t, KID_ROUTE);
     }
     float lmax = __shfl_sync(0xFFFFFFFFu, my_val, 0);
-    float p = (lane < a.k) ? expf(my_val - lmax) : 0.0f;
+    float p = (lane < k) ? expf(my_val - lmax) : 0.0f;
     float s = p;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (lane < a.k) {
-        a.ids[static_cast<size_t>(t) * a.k + lane] = my_id;
-        a.weights[static_cast<size_t>(t) * a.k + lane] = p / s;
+    if (lane < k) {
+        ids_out[lane] = my_id;
+        w_out[lane] = p / s;
     }
+}
+
+template <int NI>
+__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane) {
+    route_one<NI>(a.logits + static_cast<size_t>(t) * a.E, a.keep, a.E, a.k, t, lane,
+                  a.ids + static_cast<size_t>(t) * a.k, a.weights + static_cast<size_t>(t) * a.k, a.err);
 }
 
 // Stable grouping of all T*k entries by one CTA of kRouteWarps warps.

@@ -60,9 +60,28 @@ __global__ void fill_kernel(uint8_t* dst, Parts ps) {
     }
 }
 
+// Drop the L2 lines of a buffer without writing them back (its contents are
+// garbage): one 128-byte line per thread.
+__global__ void l2_discard_kernel(uint8_t* p, size_t lines) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < lines;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        asm volatile("discard.global.L2 [%0], 128;" ::"l"(p + 128 * i) : "memory");
+}
+
 }  // namespace
 
 extern "C" {
+
+// Benchmark helper: after a buffer larger than L2 has been written to push
+// every earlier line out of L2, discard that buffer's lines (no write-back),
+// so the next kernel starts with a cold and clean L2 instead of paying for
+// the flush buffer's dirty lines.  p 128-byte aligned, bytes a multiple of
+// 128.  Returns a cudaError_t value (0 = ok).
+int moe_synth_l2_discard(void* p, size_t bytes, void* stream) {
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 127) || (bytes & 127)) return static_cast<int>(cudaErrorInvalidValue);
+    l2_discard_kernel<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint8_t*>(p), bytes / 128);
+    return static_cast<int>(cudaGetLastError());
+}
 
 // Bytes of one expert object (same as moe_fp4_slot_bytes for a valid shape).
 size_t moe_synth_expert_bytes(int hidden, int inter) {

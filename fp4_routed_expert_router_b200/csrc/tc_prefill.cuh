@@ -17,21 +17,28 @@
 // stage (128 K, two 128-byte swizzle atoms).  One persistent CTA per SM, warp
 // roles:
 //   warps 0-15   dequantisers: warp w works in TMEM lane group w % 4 and
-//                decodes 32-K chunk w / 4 of every stage: each thread takes
-//                its row's 32 codes from the staged FP4 blocks (exact E2M1 x
-//                2^(s-127) -> bf16, fp4_decode.cuh) and writes them to the
-//                stage's A columns in TMEM with tcgen05.st (lane = row, two
-//                bf16 per column).
+//                takes lane column c = w / 4 of every 128-K stage: each
+//                thread reads its row's 16-byte chunk c (codes 8c .. 8c+7 of
+//                the four 32-K blocks, slot_layout.cuh), converts them to f16
+//                (exact E2M1), multiplies each block by 2^(s - s_ref) with
+//                s_ref the row's largest scale (exact while the row's scales
+//                span at most 24 binades: f16 reaches 2^-24), and writes them
+//                to the stage's A columns in TMEM with tcgen05.st (lane =
+//                row, two f16 per column, K in natural order).
 //   warps 16-19  epilogue: tcgen05.ld of the finished accumulator (double
-//                buffered), SwiGLU -> h (bf16) or o (fp32, scattered back to
-//                token-expert order), overlapping the next item's MMAs.
+//                buffered), times 2^(s_ref - 127) of the row and the
+//                column's 2^-sigma (B is prescaled f16), SwiGLU -> h (bf16) or
+//                o (fp32, scattered back to token-expert order), overlapping
+//                the next item's MMAs.
 //   warp 20      B producer: TMA tensor loads of the stage's 16-row boxes of
-//                gathered token rows (x grouped by expert, or h), 128-byte
+//                gathered token rows (x grouped by expert, or h, both as f16
+//                with an exact power-of-two prescale per row), 128-byte
 //                swizzle, into shared memory.
 //   warp 21      code producer: cp.async.bulk of the item's slot blocks (all
 //                of its rows for one block's K = two stages) into a ring.
-//   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A from
-//                TMEM and B from shared memory (fp32 accumulate in TMEM), eight
+//   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 (f16 x f16)
+//                with A from TMEM and B from shared memory (fp32 accumulate
+//                in TMEM), eight
 //                K=16 instructions per stage; tcgen05.commit frees the stage
 //                and, after the last stage, hands the accumulator over.
 // A stage is "full" when all 16 dequant warps have arrived and the B bytes
@@ -47,7 +54,7 @@
 #include "../../include/moe_fp4.h"
 #include "common.cuh"
 #include "decode_common.cuh"
-#include "fp4_decode.cuh"
+#include "fp4_cvt.cuh"
 #include "slot_layout.cuh"
 #include "tma.cuh"
 
@@ -65,7 +72,10 @@ constexpr int kTcAccCols = 2 * kTcNmax;   // two accumulators of kTcNmax fp32 co
 constexpr int kTcMaxEntries = 8;   // code ring entries at most
 
 struct TcArgs {
-    GemvArgs g;
+    ExpertArgs g;
+    const uint8_t* rowref;  // [n_slots][2I + H]: largest scale byte of each w1, w3, w2 row
+    const float* colscale;  // [T*k] 2^-sigma of each B row (gathered x, or h)
+    uint16_t* hb;           // [T*k, I] bf16 h (up output, grouped order)
     SlotLayout L;
     int T;
     int off_b;             // dynamic smem offset of the B ring (1024-aligned), kTcStages x 2 atoms x kTcNmax rows x 128 bytes
@@ -73,6 +83,7 @@ struct TcArgs {
     int entry_bytes;       // the item's slot blocks for one block's K (4 up / 8 down blocks)
     int centries;          // 0 when the shape does not fit
     int max_active;
+    unsigned long long timeout_ns;   // limit of each bounded wait
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -84,16 +95,15 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
            (static_cast<uint64_t>(2) << 61);
 }
 
-__device__ __forceinline__ uint32_t umma_idesc_bf16(int m, int n) {
-    // D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1), B bf16 (10-12 = 1), both
+__device__ __forceinline__ uint32_t umma_idesc_f16(int m, int n) {
+    // D fp32 (bits 4-5 = 1), A f16 (7-9 = 0), B f16 (10-12 = 0), both
     // K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
-           (static_cast<uint32_t>(m >> 4) << 24);
+    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-// One tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128) with A read from
-// tensor memory (lane = row, two bf16 per column) and B from shared memory.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+// One tcgen05.mma (kind::f16, f16 x f16 -> fp32, M = 128) with A read from
+// tensor memory (lane = row, two f16 per column) and B from shared memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -130,6 +140,21 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 4 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st4_nowait(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
+                 "r"(r3)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// f16x2 product (exact here: a power of two times an E2M1 value).
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -139,17 +164,49 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 }
 
 // ------------------------------------------------------------------ gather
-// x rows in grouped (expert-major) order: xg[p] = x[perm[p] / k].
+// Token rows in grouped (expert-major) order as prescaled f16 (fp4_cvt.cuh):
+// xg[p] = x[perm[p] / k] * 2^sigma, colscale[p] = 2^-sigma, sigma from the
+// row's largest |x|.  One CTA per grouped row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* x, const int32_t* perm, int k, int H,
-                                                          int n_rows, uint16_t* xg) {
+                                                          int n_rows, uint16_t* xg, float* colscale) {
+    __shared__ uint32_t red[8];
     pdl_wait();
     pdl_trigger();
     const int row = blockIdx.x;
     if (row >= n_rows) return;
     const int src = __ldg(perm + row) / k;
-    const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<size_t>(src) * H);
-    uint4* d = reinterpret_cast<uint4*>(xg + static_cast<size_t>(row) * H);
-    for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d[i] = s[i];
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(src) * H);
+    uint32_t mx = 0;
+    for (int i = threadIdx.x; i < H / 2; i += blockDim.x) mx = max(mx, bf16x2_absmax(s[i]));
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    uint32_t tot = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot = max(tot, red[w]);
+    const int sg = prescale_sigma(tot);
+    const float mult = pow2i(sg);
+    uint32_t* d = reinterpret_cast<uint32_t*>(xg + static_cast<size_t>(row) * H);
+    for (int i = threadIdx.x; i < H / 2; i += blockDim.x) d[i] = bf16x2_scaled_to_f16x2(s[i], mult);
+    if (threadIdx.x == 0) colscale[row] = pow2i(-sg);
+}
+
+// h rows (bf16, grouped order) -> prescaled f16 for the down GEMM: one warp
+// per row, sigma from the row's largest |h|.
+__global__ void __launch_bounds__(256) h_convert_kernel(const uint16_t* hb, int I, int n_rows, uint16_t* hh,
+                                                        float* colscale) {
+    pdl_wait();
+    pdl_trigger();
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (row >= n_rows) return;
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(hb + static_cast<size_t>(row) * I);
+    uint32_t mx = 0;
+    for (int i = lane; i < I / 2; i += 32) mx = max(mx, bf16x2_absmax(__ldcg(s + i)));
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    const int sg = prescale_sigma(mx);
+    const float mult = pow2i(sg);
+    uint32_t* d = reinterpret_cast<uint32_t*>(hh + static_cast<size_t>(row) * I);
+    for (int i = lane; i < I / 2; i += 32) d[i] = bf16x2_scaled_to_f16x2(__ldcg(s + i), mult);
+    if (lane == 0) colscale[row] = pow2i(-sg);
 }
 
 // ------------------------------------------------------------------ GEMM
@@ -166,7 +223,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     // the 128-byte swizzle of the B tiles is defined on 1024-byte atoms of the
     // shared address space: align the working base explicitly
     uint8_t* smem = tc_smem_raw + ((1024u - (smem_u32(tc_smem_raw) & 1023u)) & 1023u);
-    const GemvArgs& a = t.g;
+    const ExpertArgs& a = t.g;
     const SlotLayout& L = t.L;
     const int CE = t.centries;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // A decoded + B landed
@@ -175,7 +232,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     uint64_t* cfree = cfull + CE;
     uint64_t* acc_full = cfree + CE;             // [2]
     uint64_t* acc_empty = acc_full + 2;          // [2]
-    Fp4Lut* lut = reinterpret_cast<Fp4Lut*>(smem + 1024);              // 4 KB, 16-byte aligned
+    uint32_t* mtab = reinterpret_cast<uint32_t*>(smem + 1024);          // f16x2 2^-i, i = 0..255 (4 KB reserved)
     int* act_e = reinterpret_cast<int*>(smem + 1024 + 256 * 16);
     int* act_p0 = act_e + t.max_active;
     int* act_m = act_p0 + t.max_active;
@@ -218,7 +275,10 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                      "r"(512u));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    for (int i = tid; i < 256; i += blockDim.x) lut[i] = make_fp4_lut(static_cast<uint32_t>(i));
+    for (int i = tid; i < 256; i += blockDim.x) {   // 2^-i as f16 (subnormal from 2^-15 to 2^-24, then 0)
+        const uint32_t hb16 = i <= 14 ? static_cast<uint32_t>(15 - i) << 10 : (i <= 24 ? 1u << (24 - i) : 0u);
+        mtab[i] = hb16 | (hb16 << 16);
+    }
     pdl_wait();
     {   // active experts and the prefix of their work items
         int* offs_s = scratch;
@@ -290,10 +350,10 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
 
     if (warp < kTcDequantWarps) {
         // ------------------------------------------------------------ dequantisers
-        // Warp w works in TMEM lane group w % 4 and decodes 32-K chunk w / 4 of
-        // every stage (four chunks per 128-K stage) for the 32 rows of its
-        // lanes, into the stage's A columns with one tcgen05.st.
-        const int ch = warp >> 2;                              // chunk of the stage
+        // Warp w works in TMEM lane group w % 4 and lane column c = w / 4:
+        // per 128-K stage each thread converts its row's chunk c (eight codes
+        // of each of the four 32-K blocks) and stores four 4-column pieces.
+        const int cc = warp >> 2;                              // lane column of the stage
         const int rr = lane & 15;                              // row inside the slot block
         const int blk = UP ? lg : 2 * lg + (lane >> 4);        // slot block of the entry
         const int mat = UP ? (lane >> 4) : 0;                  // w1 / w3 half of an up block
@@ -305,29 +365,36 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             item_of(i, ai, mt, n0);
             const int slot = act_slot[ai];
             if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[ai], kid);
+            // the row's largest scale (load-time table)
+            const int wrow = UP ? (mt * ROWT + lg) * 16 + rr : (mt * ROWT + blk) * 16 + rr;
+            const int sref = slot < 0 ? 0
+                                      : __ldg(t.rowref + static_cast<size_t>(slot) * (2 * a.I + a.H) +
+                                              (UP ? mat * a.I : 2 * a.I) + wrow);
             for (int f = 0; f < nfb; ++f, ++gentry) {
                 const int ce = gentry % CE;
-                if (!mbar_wait(&cfull[ce], (gentry / CE) & 1, abort_flag) && lane == 0)
+                if (!mbar_wait(&cfull[ce], (gentry / CE) & 1, abort_flag, t.timeout_ns) && lane == 0)
                     latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
                 const uint8_t* ent = code_entry(ce);
                 for (int j = 0; j < spe; ++j, ++gstg) {
                     const int st = gstg % S;
-                    if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag) && lane == 0)
+                    if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
                         latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
                     tc_fence_after();
-                    const int q = 4 * j + ch;                   // 32-K chunk of the block row
-                    const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off + swizzle_chunk(q, rr, rbb) * 16);
-                    const Fp4Lut lt = lut[ent[scale_off + q]];
-                    uint32_t o[16];
-                    fp4_decode8(w.x, lt, o);
-                    fp4_decode8(w.y, lt, o + 4);
-                    fp4_decode8(w.z, lt, o + 8);
-                    fp4_decode8(w.w, lt, o + 12);
-                    if (slot < 0) {
+                    // stage j = 128-K group j of the block row
+                    const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off +
+                                                                    swizzle_chunk(4 * j + cc, rr, rbb) * 16);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t*>(ent + scale_off + 4 * j);
+                    const uint32_t col0 = tmem_a + lane_addr + st * ACOLS + 4 * cc;
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) o[c] = 0;
+                    for (int q = 0; q < 4; ++q) {   // 32-K block q of the group: K = 32q + 8cc .. +7
+                        const int sq = static_cast<int>(__byte_perm(sw, 0u, 0x4440u | static_cast<uint32_t>(q)));
+                        const uint32_t mult = (slot < 0) ? 0u : mtab[(sref - sq) & 255];
+                        uint32_t o[4];
+                        e2m1x8_to_f16x2(q == 0 ? w.x : q == 1 ? w.y : q == 2 ? w.z : w.w, o);
+                        tmem_st4_nowait(col0 + 16 * q, hmul2_u32(o[0], mult), hmul2_u32(o[1], mult),
+                                        hmul2_u32(o[2], mult), hmul2_u32(o[3], mult));
                     }
-                    tmem_st16(tmem_a + lane_addr + st * ACOLS + ch * 16, o);
+                    tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full[st]);
@@ -344,9 +411,16 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             const int p0 = act_p0[ai], m = act_m[ai], slot = act_slot[ai];
             const int nvalid = min(kTcNmax, m - n0);
             const int ab = i & 1;
-            if (!mbar_wait(&acc_full[ab], (i >> 1) & 1, abort_flag) && lane == 0)
+            if (!mbar_wait(&acc_full[ab], (i >> 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
                 latch_error(a.err, ERR_ETIMEOUT, i, kid);
             tc_fence_after();
+            // this lane's weight row and its 2^(s_ref - 127)
+            const int erow = UP ? (mt * ROWT + lg) * 16 + (lane & 15) : mt * OUT_ROWS + 32 * lg + lane;
+            const int emat = UP ? (lane >> 4) : 2;
+            const float rowmul = slot < 0 ? 0.0f
+                                          : pow2i(static_cast<int>(__ldg(t.rowref + static_cast<size_t>(slot) *
+                                                                                        (2 * a.I + a.H) +
+                                                                         emat * a.I + erow)) - 127);
             for (int c16 = 0; c16 * 16 < nvalid; ++c16) {
                 uint32_t v[16];
                 tmem_ld16(tmem + lane_addr + ab * kTcNmax + c16 * 16, v);
@@ -354,12 +428,14 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                     // lanes 0-15: a1 of rows 16 lg + lane; lanes 16-31 hold the matching a3
 #pragma unroll
                     for (int qq = 0; qq < 16; ++qq) {
-                        const float a3 = __uint_as_float(__shfl_down_sync(0xFFFFFFFFu, v[qq], 16));
                         const int jt = c16 * 16 + qq;
+                        const float cs = (jt < nvalid) ? __ldg(t.colscale + p0 + n0 + jt) : 0.0f;
+                        const float mine = __uint_as_float(v[qq]) * rowmul * cs;
+                        const float a3 = __shfl_down_sync(0xFFFFFFFFu, mine, 16);
                         if (lane < 16 && jt < nvalid) {
-                            const float a1 = __uint_as_float(v[qq]);
+                            const float a1 = mine;
                             const float hv = (slot >= 0) ? a1 / (1.0f + expf(-a1)) * a3 : 0.0f;
-                            a.hbuf[static_cast<size_t>(p0 + n0 + jt) * a.I + mt * OUT_ROWS + 16 * lg + lane] =
+                            t.hb[static_cast<size_t>(p0 + n0 + jt) * a.I + mt * OUT_ROWS + 16 * lg + lane] =
                                 f32_to_bf16_rne(hv);
                         }
                     }
@@ -369,8 +445,9 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                         const int jt = c16 * 16 + qq;
                         if (jt < nvalid) {
                             const int entn = __ldg(a.perm + p0 + n0 + jt);
+                            const float cs = __ldg(t.colscale + p0 + n0 + jt);
                             a.obuf[static_cast<size_t>(entn) * a.H + mt * OUT_ROWS + 32 * lg + lane] =
-                                (slot >= 0) ? __uint_as_float(v[qq]) : 0.0f;
+                                (slot >= 0) ? __uint_as_float(v[qq]) * rowmul * cs : 0.0f;
                         }
                     }
                 }
@@ -382,8 +459,11 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     } else if (warp == kTcDequantWarps + kTcEpiWarps) {
         // ------------------------------------------------------------ B producer
         // The whole warp walks the loop (warp-uniform waits); lane 0 issues.
+        // After a wait gives up no further copy is issued (a stage is never
+        // the target of two copies at once); the decision is warp-uniform.
         int gstg = 0;
-        for (int i = 0; i < my_items; ++i) {
+        bool stop = false;
+        for (int i = 0; i < my_items && !stop; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int nvalid = min(kTcNmax, act_m[ai] - n0);
@@ -391,8 +471,13 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             const int row0 = act_p0[ai] + n0;
             for (int s = 0; s < n_stg; ++s, ++gstg) {
                 const int st = gstg % S;
-                if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                int ok = 1;
+                if (gstg >= S && lane == 0) ok = mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns);
+                if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                    if (lane == 0) latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                    stop = true;
+                    break;
+                }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(2 * nb * 16 * 128));
                     for (int at = 0; at < 2; ++at)
@@ -415,7 +500,8 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
         // ------------------------------------------------------------ code producer (FP4 blocks)
         const uint64_t pol = policy_evict_first();
         int gentry = 0;
-        for (int i = 0; i < my_items; ++i) {
+        bool stop = false;
+        for (int i = 0; i < my_items && !stop; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int slot = act_slot[ai];
@@ -423,8 +509,14 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                                  (UP ? 0 : L.up_bytes);
             for (int f = 0; f < nfb; ++f, ++gentry) {
                 const int ce = gentry % CE;
-                if (gentry >= CE && !mbar_wait(&cfree[ce], ((gentry / CE) - 1) & 1, abort_flag) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
+                int ok = 1;
+                if (gentry >= CE && lane == 0)
+                    ok = mbar_wait(&cfree[ce], ((gentry / CE) - 1) & 1, abort_flag, t.timeout_ns);
+                if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                    if (lane == 0) latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
+                    stop = true;
+                    break;
+                }
                 if (lane == 0) {
                     if (slot < 0) {
                         mbar_arrive(&cfull[ce]);
@@ -456,15 +548,15 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             item_of(i, ai, mt, n0);
             const int nvalid = min(kTcNmax, act_m[ai] - n0);
             const int n = (nvalid + 15) / 16 * 16;
-            const uint32_t idesc = umma_idesc_bf16(kTcM, n);
+            const uint32_t idesc = umma_idesc_f16(kTcM, n);
             const int ab = i & 1;
-            if (i >= 2 && !mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, abort_flag) && lane == 0)
+            if (i >= 2 && !mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
                 latch_error(a.err, ERR_ETIMEOUT, i, kid);
             tc_fence_after();
             const uint32_t dacc = tmem + ab * kTcNmax;
             for (int s = 0; s < n_stg; ++s, ++gstg) {
                 const int st = gstg % S;
-                if (!mbar_wait(&full[st], (gstg / S) & 1, abort_flag) && lane == 0)
+                if (!mbar_wait(&full[st], (gstg / S) & 1, abort_flag, t.timeout_ns) && lane == 0)
                     latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
                 tc_fence_after();
                 const uint64_t bdesc = umma_desc_sw128(smem_u32(stage_b(st)));
@@ -474,7 +566,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                     for (int at = 0; at < 2; ++at)
 #pragma unroll
                         for (int kk = 0; kk < kTcBK / 16; ++kk)   // K = 16: 8 TMEM columns of A, +32 bytes of B
-                            umma_bf16_ts(dacc, acol + at * (kTcBK / 2) + 8 * kk,
+                            umma_f16_ts(dacc, acol + at * (kTcBK / 2) + 8 * kk,
                                          bdesc + static_cast<uint64_t>((at * BATOM) >> 4) + 2 * kk, idesc,
                                          (s > 0 || at > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sfree[st]);                  // stage reusable once these MMAs are done
@@ -499,9 +591,13 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
 // ------------------------------------------------------------------ host side
 struct TcPlan {
     int ready;
-    uint16_t* xg;          // gathered x rows [max_tokens * k, H]
-    CUtensorMap map_x;     // bf16 [rows, H], box {64, 16}, 128-byte swizzle
-    CUtensorMap map_h;     // bf16 [rows, I], box {64, 16}, 128-byte swizzle
+    uint16_t* xg;          // gathered x rows, prescaled f16 [max_tokens * k, H]
+    float* xcs;            // [max_tokens * k] 2^-sigma of each gathered x row
+    uint16_t* hb;          // h, bf16 [max_tokens * k, I] (up output)
+    uint16_t* hh;          // h, prescaled f16 [max_tokens * k, I] (down input; owned by the context)
+    float* hcs;            // [max_tokens * k] 2^-sigma of each h row
+    CUtensorMap map_x;     // f16 [rows, H], box {64, 16}, 128-byte swizzle
+    CUtensorMap map_h;     // f16 [rows, I], box {64, 16}, 128-byte swizzle
     int rows;
     int smem_limit;
     int sm_count;
@@ -520,20 +616,26 @@ inline bool tc_encode_map(CUtensorMap* map, void* base, int rows, int cols) {
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcBK), 16};
     const cuuint32_t estr[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline cudaError_t tc_plan_create(TcPlan* p, const moe_fp4_config& cfg, uint16_t* hbuf, int sm_count,
+inline cudaError_t tc_plan_create(TcPlan* p, const moe_fp4_config& cfg, uint16_t* hh, int sm_count,
                                   int smem_limit) {
     *p = TcPlan{};
     p->rows = cfg.max_tokens * cfg.top_k;
     p->sm_count = sm_count;
     p->smem_limit = smem_limit;
-    cudaError_t e = cudaMalloc(&p->xg, sizeof(uint16_t) * static_cast<size_t>(p->rows) * cfg.hidden);
-    if (e != cudaSuccess) return e;
-    if (!tc_encode_map(&p->map_x, p->xg, p->rows, cfg.hidden) || !tc_encode_map(&p->map_h, hbuf, p->rows, cfg.inter))
+    p->hh = hh;
+    const size_t rows = static_cast<size_t>(p->rows);
+    cudaError_t e;
+    if ((e = cudaMalloc(&p->xg, sizeof(uint16_t) * rows * cfg.hidden)) != cudaSuccess ||
+        (e = cudaMalloc(&p->xcs, sizeof(float) * rows)) != cudaSuccess ||
+        (e = cudaMalloc(&p->hb, sizeof(uint16_t) * rows * cfg.inter)) != cudaSuccess ||
+        (e = cudaMalloc(&p->hcs, sizeof(float) * rows)) != cudaSuccess)
+        return e;
+    if (!tc_encode_map(&p->map_x, p->xg, p->rows, cfg.hidden) || !tc_encode_map(&p->map_h, hh, p->rows, cfg.inter))
         return cudaErrorInvalidValue;
     auto set = [&](const void* f) {
         return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_limit);
@@ -546,7 +648,11 @@ inline cudaError_t tc_plan_create(TcPlan* p, const moe_fp4_config& cfg, uint16_t
 
 inline void tc_plan_destroy(TcPlan* p) {
     if (p->xg) cudaFree(p->xg);
-    p->xg = nullptr;
+    if (p->xcs) cudaFree(p->xcs);
+    if (p->hb) cudaFree(p->hb);
+    if (p->hcs) cudaFree(p->hcs);
+    p->xg = p->hb = nullptr;
+    p->xcs = p->hcs = nullptr;
     p->ready = 0;
 }
 
@@ -558,9 +664,13 @@ inline bool tc_prefers(int T, const moe_fp4_config& cfg) {
     return 4LL * T * cfg.top_k >= 3LL * cfg.n_experts;
 }
 
-inline TcArgs tc_args(const TcPlan& p, const GemvArgs& g, const SlotLayout& L, int T, bool up) {
+inline TcArgs tc_args(const TcPlan& p, const ExpertArgs& g, const SlotLayout& L, int T, bool up,
+                      const uint8_t* rowref) {
     TcArgs t{};
     t.g = g;
+    t.rowref = rowref;
+    t.colscale = up ? p.xcs : p.hcs;
+    t.hb = p.hb;
     t.L = L;
     t.T = T;
     const int ent = T * g.k;

@@ -50,15 +50,29 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 }
 
 // One bounded probe of phase `parity`: the hardware may suspend the thread
-// for up to ~0.5 ms waiting for the phase (instead of a hot spin).
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// for up to `hint_ns` (at most ~0.5 ms) waiting for the phase instead of a
+// hot spin.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns = 500000u) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking probe: has phase `parity` of `bar` completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -75,9 +89,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // a broken pipeline costs one timeout, not one per item.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns = 1000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t hint = timeout_ns < 500000ull ? static_cast<uint32_t>(timeout_ns) : 500000u;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait(bar, parity, hint)) {
         if (*abort) return false;
         if (global_timer_ns() - t0 > timeout_ns) {
             *abort = 1;

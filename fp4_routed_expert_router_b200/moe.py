@@ -19,12 +19,14 @@ SYNTH_PATH = os.path.join(_PKG, "lib", "libmoe_synth.so")
 OK, EINVAL, ENOMEM, ECUDA, ESLOT, ETIMEOUT = 0, 1, 2, 3, 4, 5
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOMEM", 3: "ECUDA", 4: "ESLOT", 5: "ETIMEOUT"}
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
-OPT_PATH, OPT_PROFILE = 1, 2
+OPT_PATH, OPT_PROFILE, OPT_WAIT_LIMIT_US = 1, 2, 3
 
 # every symbol include/moe_fp4.h declares
 EXPORTS = ("moe_fp4_slot_bytes", "moe_fp4_create", "moe_fp4_destroy", "moe_fp4_arena",
            "moe_fp4_set_option", "moe_fp4_profile_read", "moe_fp4_load_expert_slot", "moe_fp4_route",
-           "moe_fp4_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc", "moe_fp4_saliency", "moe_fp4_stream_experts", "moe_fp4_residency_stats", "moe_fp4_expert_outputs", "moe_fp4_combine")
+           "moe_fp4_forward", "moe_fp4_route_forward", "moe_fp4_last_error", "moe_fp4_forward_noalloc",
+           "moe_fp4_saliency", "moe_fp4_stream_experts", "moe_fp4_residency_stats", "moe_fp4_expert_outputs",
+           "moe_fp4_combine")
 
 
 class MoeError(RuntimeError):
@@ -69,6 +71,8 @@ def load(path: str = LIB_PATH):
         L.moe_fp4_route.argtypes = [P, I32, P, P, I32, P, P, P, P, P, P]
         L.moe_fp4_forward.restype = I32
         L.moe_fp4_forward.argtypes = [P, I32, P, I32, P, P, P, P, P, P, P, P]
+        L.moe_fp4_route_forward.restype = I32
+        L.moe_fp4_route_forward.argtypes = [P, I32, P, P, P, I32, P, P, P, P, P, P, P, P]
         L.moe_fp4_saliency.restype = I32
         L.moe_fp4_saliency.argtypes = [P, I32, P, P, P, P, P]
         L.moe_fp4_stream_experts.restype = I32
@@ -95,6 +99,8 @@ def load_synth(path: str = SYNTH_PATH):
         S = ctypes.CDLL(path)
         S.moe_synth_expert_bytes.restype = ctypes.c_size_t
         S.moe_synth_expert_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+        S.moe_synth_l2_discard.restype = ctypes.c_int
+        S.moe_synth_l2_discard.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         S.moe_synth_fill_expert.restype = ctypes.c_int
         S.moe_synth_fill_expert.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -122,6 +128,17 @@ def synth_fill_expert(dst: torch.Tensor, seed: int, layer: int, expert: int, hid
                                             scale_lo, scale_hi, _stream(stream))
     if rc != 0:
         raise RuntimeError(f"moe_synth_fill_expert failed: cuda error {rc}")
+
+
+def l2_flush(buf: torch.Tensor, value: float = 0.0, stream=None) -> None:
+    """Push every earlier line out of L2 by writing ``buf`` (larger than L2),
+    then drop ``buf``'s own lines without write-back: the next kernel starts
+    with a cold, clean L2."""
+    buf.fill_(value)
+    n = buf.numel() * buf.element_size() // 128 * 128
+    rc = load_synth().moe_synth_l2_discard(_ptr(buf), n, _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"moe_synth_l2_discard failed: cuda error {rc}")
 
 
 @dataclass
@@ -181,6 +198,10 @@ class Context:
 
     def set_path(self, path: int) -> None:
         self._check(self.lib.moe_fp4_set_option(self.h, OPT_PATH, path), "set_option")
+
+    def set_wait_limit_us(self, us: int) -> None:
+        """Limit of every bounded device-side wait (0 restores the default, 1 s)."""
+        self._check(self.lib.moe_fp4_set_option(self.h, OPT_WAIT_LIMIT_US, int(us)), "set_option")
 
     def set_profile(self, on: bool) -> None:
         self._check(self.lib.moe_fp4_set_option(self.h, OPT_PROFILE, 1 if on else 0), "set_option")
@@ -245,6 +266,19 @@ class Context:
         self._check(rc, "forward")
         return y
 
+    def route_forward(self, layer: int, logits: torch.Tensor, x: torch.Tensor, keep: torch.Tensor | None = None,
+                      out: Routing | None = None, y: torch.Tensor | None = None,
+                      x_out: torch.Tensor | None = None, stream=None) -> tuple[Routing, torch.Tensor]:
+        """Route + forward in one call (one kernel for decode batches)."""
+        T = x.shape[0]
+        r = out if out is not None else self.alloc_routing(T)
+        if y is None:
+            y = torch.empty((T, self.cfg.hidden), dtype=torch.float32, device=x.device)
+        rc = self.lib.moe_fp4_route_forward(self.h, layer, _ptr(logits), _ptr(keep), _ptr(x), T, _ptr(r.ids),
+                                            _ptr(r.weights), _ptr(r.counts), _ptr(r.offsets), _ptr(r.perm),
+                                            _ptr(y), _ptr(x_out), _stream(stream))
+        self._check(rc, "route_forward")
+        return r, y
 
     def expert_outputs(self, layer: int, x: torch.Tensor, experts: torch.Tensor, o: torch.Tensor | None = None,
                        stream=None) -> torch.Tensor:

@@ -32,10 +32,10 @@
  *
  * Calls: slot_bytes, create, destroy, arena, set_option, profile_read (the
  * context); load_expert_slot, stream_experts, residency_stats (the arena);
- * route, forward, last_error (the layer); expert_outputs, combine (the two
- * halves of forward, for expert-parallel use); saliency (per-expert
- * statistic of the last forward); forward_noalloc (forward without any
- * allocation, library-owned static scratch).
+ * route, forward, route_forward, last_error (the layer); expert_outputs,
+ * combine (the two halves of forward, for expert-parallel use); saliency
+ * (per-expert statistic of the last forward); forward_noalloc (forward
+ * without any allocation, library-owned static scratch).
  */
 #ifndef MOE_FP4_H
 #define MOE_FP4_H
@@ -70,14 +70,20 @@ typedef struct {
 
 /* Execution-path override for moe_fp4_set_option(MOE_FP4_OPT_PATH, .). */
 enum {
-    MOE_FP4_PATH_AUTO = 0,  /* grouped GEMV while 4*T*k < 3*E, tcgen05 GEMM from there on */
-    MOE_FP4_PATH_GEMV = 1,  /* always the register-decoded grouped GEMV */
+    MOE_FP4_PATH_AUTO = 0,  /* decode kernel while 4*T*k < 3*E, tcgen05 GEMM from there on */
+    MOE_FP4_PATH_GEMV = 1,  /* always the decode kernel (grouped mma.sync GEMV) */
     MOE_FP4_PATH_TC = 2     /* always the tcgen05 grouped GEMM */
 };
 /* Options for moe_fp4_set_option. */
 enum {
-    MOE_FP4_OPT_PATH = 1,     /* value: MOE_FP4_PATH_* */
-    MOE_FP4_OPT_PROFILE = 2   /* value 1: time every kernel with CUDA events */
+    MOE_FP4_OPT_PATH = 1,          /* value: MOE_FP4_PATH_* */
+    MOE_FP4_OPT_PROFILE = 2,       /* value 1: time every kernel with CUDA events */
+    MOE_FP4_OPT_WAIT_LIMIT_US = 3  /* value: limit of every bounded device-side wait of the
+                                      layer kernels in microseconds (1 .. 10,000,000; 0 restores
+                                      the default of 1 s).  A wait that runs out latches
+                                      MOE_FP4_ETIMEOUT; the kernel then skips its remaining waits,
+                                      lets its copies in flight land and returns (its outputs are
+                                      not valid).  The context stays usable. */
 };
 
 /*
@@ -94,13 +100,15 @@ enum {
  *      [w1 16 rows x KBu/2][w3 16 rows x KBu/2][s1 16 x KBu/32][s3 16 x KBu/32]
  *  then down blocks, for each 16-row tile of W2 and each K block of KBd
  *  (256 when it divides I, else 128):  [w2 16 rows x KBd/2][s2 16 x KBd/32]
- * so one 16-row tile of w1+w3 over all of H (87,040 bytes for V4.1) and 32
- * rows of w2 over all of I (39,168 bytes) are each contiguous.  In code rows
- * of 128-byte multiples the 16-byte chunk q of row r sits at
- * q ^ ((r & 7) ^ ((r & 1) << 2)) (bank-conflict-free loads), and each 32-bit
- * code word is re-encoded (the eight sign bits move so that the in-register
- * decoder of csrc/fp4_decode.cuh needs fewer instructions; magnitudes stay in
- * place).  Scale bytes are stored as they are.  The total is unchanged.
+ * so one 16-row x KBu block of w1+w3 (4,352 bytes for V4.1) and 16 rows of
+ * w2 over all of I (19,584 bytes) are each contiguous.  Code bytes keep the
+ * checkpoint's nibbles, but inside each 64-byte group of a row (128 K = four
+ * 32-K scale blocks) the sixteen 32-bit words are transposed: 16-byte chunk c
+ * holds, as its word j, codes K = 32j + 8c .. +7 of the group, which hands one
+ * MMA lane column eight codes of each scale block.  In code rows of 128-byte
+ * multiples the 16-byte chunk q of row r sits at q ^ ((r & 7) ^ ((r & 1) << 2))
+ * (bank-conflict-free loads).  Scale bytes are stored as they are.  The total
+ * is unchanged.
  */
 size_t moe_fp4_slot_bytes(const moe_fp4_config *cfg);
 
@@ -111,8 +119,10 @@ size_t moe_fp4_slot_bytes(const moe_fp4_config *cfg);
  *               NULL, in which case the library allocates (and frees) it.
  *  arena_bytes: size of a caller arena (ignored when arena is NULL).
  * The library also allocates the slot table (int32 [L][E], every entry -1 =
- * unmapped), a staging buffer of one slot, a workspace sized from max_tokens
- * and a device error word.  On failure *out is NULL and nothing is leaked.
+ * unmapped), a table of each slot's largest scale byte per weight row
+ * (n_slots * (2I + H) bytes), a staging buffer of one slot, a workspace sized
+ * from max_tokens and a device error word.  On failure *out is NULL and
+ * nothing is leaked.
  * Errors: EINVAL (bad config / pointers), ENOMEM, ECUDA.
  */
 moe_fp4_status moe_fp4_create(const moe_fp4_config *cfg, int device, void *arena,
@@ -152,8 +162,9 @@ int moe_fp4_profile_read(moe_fp4_ctx *ctx, const char **names, float *ms, int ma
  * Whatever was mapped to `slot` before is unmapped; a previous slot of
  * (layer, expert) is released.  slot = -1 only unmaps (layer, expert) and the
  * pointers are ignored.  Supported scale bytes are 2..252 (every value whose
- * E2M1 multiples are normal bf16 numbers); others latch EINVAL in the error
- * word.  Errors: EINVAL (indices, NULL tensors), ECUDA.
+ * block multiplier 2^(s-127) is a normal fp32 number and whose E2M1 multiples
+ * are normal bf16 numbers); others latch EINVAL in the error word.  Errors:
+ * EINVAL (indices, NULL tensors), ECUDA.
  */
 moe_fp4_status moe_fp4_load_expert_slot(moe_fp4_ctx *ctx, int layer, int expert, int slot,
                                         const uint8_t *w1, const uint8_t *w1_scale,
@@ -220,8 +231,13 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx *ctx, int layer, const float *logits,
  *  x_out     bf16 [T, H] out or NULL, 8-byte aligned: bf16_rne(x + y), the
  *            residual update of a stacked layer; may alias x.
  * An entry routed to an expert with no slot contributes zero and latches
- * ESLOT.  Scratch (the bf16 h rows and per-entry fp32 outputs) lives in the
- * context's workspace, so calls on one context must not overlap in time.
+ * ESLOT.  Scratch (prescaled x and h rows, per-entry fp32 outputs and the
+ * decode kernel's barrier counters) lives in the context's workspace, so calls
+ * on one context must not overlap in time.
+ * Path: while 4*T*k < 3*E one persistent kernel runs the
+ * whole layer -- w1/w3 GEMV with SwiGLU, w2 GEMV and, for T <= 16, the
+ * combine -- with one CTA per SM launched cooperatively; larger batches run
+ * the tcgen05 grouped GEMMs.  MOE_FP4_OPT_PATH overrides the choice.
  * Errors: EINVAL, ECUDA.
  */
 moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, int T,
@@ -230,13 +246,28 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, i
                                const int32_t *perm, float *y, uint16_t *x_out, void *stream);
 
 /*
+ * Route and forward in one call: moe_fp4_route followed by moe_fp4_forward
+ * with the same arguments (all outputs of both are written).  For decode
+ * batches (T*k <= 64, T <= 16, E <= 384, on the decode path) the routing runs
+ * inside the layer kernel -- every CTA routes the tokens itself and the first
+ * writes ids, weights, counts, offsets and perm -- so the whole layer is one
+ * kernel launch.  Results are identical to the two calls.
+ * Errors: EINVAL, ECUDA (as route and forward).
+ */
+moe_fp4_status moe_fp4_route_forward(moe_fp4_ctx *ctx, int layer, const float *logits,
+                                     const uint8_t *keep_mask, const uint16_t *x, int T,
+                                     int32_t *ids, float *weights, int32_t *counts, int32_t *offsets,
+                                     int32_t *perm, float *y, uint16_t *x_out, void *stream);
+
+/*
  * The expert FFN for an arbitrary list of (row, expert) pairs of `layer`:
  *   o[i] = expert_{experts[i]}(x[i])   (fp32 [n, H], no router weight)
  * This is the work an expert-parallel rank does for the entries other ranks
  * dispatch to the experts it holds (moe_fp4_forward = route + this for every
  * (token, selected expert) pair + moe_fp4_combine).  The entries are grouped
- * by expert with the route kernels' stable grouping, then run on the GEMV
- * path, or on the tcgen05 path when 4n >= 3E (or as MOE_FP4_OPT_PATH forces).
+ * by expert with the route kernels' stable grouping, then run on the decode
+ * kernel, or on the tcgen05 path when 4n >= 3E (or as
+ * MOE_FP4_OPT_PATH forces).
  * Entries are processed in the same per-expert order as moe_fp4_forward
  * processes (token, slot) entries, so listing a forward's entries in
  * (token, slot) order reproduces its per-entry outputs bit for bit.
@@ -291,23 +322,28 @@ moe_fp4_status moe_fp4_saliency(moe_fp4_ctx *ctx, int T, const float *weights,
 moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
 
 /*
- * Forward without any allocation: the same decode path as moe_fp4_forward
- * (grouped GEMV, SwiGLU, combine; always the GEMV kernels), for callers that
- * cannot call cudaMalloc -- for example a plugin inside a host framework that
- * owns all device memory and forbids allocation on its execution path, or
- * code that runs where the CUDA allocator must not be entered.  This call has
- * no counterpart on the pages: it is a deployment variant of this library.
+ * Forward without any allocation: the same decode kernel as moe_fp4_forward
+ * (the whole layer in one launch: grouped GEMV, SwiGLU, combine), for callers
+ * that cannot call cudaMalloc -- for example a plugin inside a host framework
+ * that owns all device memory and forbids allocation on its execution path,
+ * or code that runs where the CUDA allocator must not be entered.  This call
+ * has no counterpart on the pages: it is a deployment variant of this library.
  *
  * Nothing is allocated and no context is used.  The caller passes every input
- * and output; the two scratch tensors of the forward (bf16 h rows and fp32
- * per-entry outputs) live in one library-owned, file-scope device array of
- * 16 MiB (16,777,216 bytes) that every GPU which loads the library holds until
- * the process exits.  A call needs T*k*(2*I + 4*H) bytes of it (the h part
- * rounded up to 256); larger T returns EINVAL before any launch.  For the
- * V4.1 shape that allows T*k <= 668 (T <= 111 at k = 6).
+ * and output; the forward's scratch (prescaled f16 x and h rows with their
+ * scales, fp32 per-entry outputs, the combine counters) lives in one
+ * library-owned, file-scope device array of 16 MiB (16,777,216 bytes) that
+ * every GPU which loads the library holds until the process exits, next to
+ * 16 bytes of grid-barrier state.  The scratch must hold
+ *   T*H*2 + T*4 + T*k*I*2 + T*k*(I/32)*4 + T*k*H*4 + (H/32)*4 bytes
+ * (each part rounded up to 256); a larger T, or a shape the decode kernel
+ * does not take, returns EINVAL before any launch.  For the V4.1 shape (k = 6)
+ * that allows T <= 103.  Up to 16 tokens the combine runs inside the kernel,
+ * above that a second kernel.
  *
- * Every call, on every stream, shares that one array and leaves the last
- * call's contents in it; nothing in it needs to start at zero.  Calls whose
+ * Every call, on every stream, shares that array and leaves the last call's
+ * contents in it; the kernel itself clears what must start at zero (the
+ * combine counters) and leaves the barrier state at zero.  Calls whose
  * executions overlap on the GPU race on it: serialise them (one stream, or
  * events).  The first call on a device looks up the array's device address
  * with cudaGetSymbolAddress (once per device, that device current); make that
@@ -317,15 +353,15 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
  *              only bound the indices used).
  *  arena       device, n_slots slots of moe_fp4_slot_bytes(cfg) bytes in the
  *              library's slot layout (as filled by moe_fp4_load_expert_slot,
- *              e.g. the arena of a context created elsewhere).
+ *              e.g. the arena of a context created elsewhere), 256-byte aligned.
  *  slot_table  device int32 [n_layers][E]: slot of (layer, expert) or -1.
  *  x, weights, offsets, perm, y, x_out, T, layer: as for moe_fp4_forward
- *              (ids and counts are not needed).
- *  err         device int32 [4] or NULL: first error latched by the kernels
+ *              (ids and counts are not needed); weights 4-byte aligned.
+ *  err         device int32 [4] or NULL: first error latched by the kernel
  *              ([0] status, [1] detail), as moe_fp4_last_error reports them;
  *              the caller clears it.  With NULL, kernel-found errors are
  *              dropped.
- * Errors: EINVAL (arguments, T beyond the scratch limit), ECUDA.
+ * Errors: EINVAL (arguments, T beyond the limits), ECUDA.
  */
 moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config *cfg, const uint8_t *arena,
                                        const int32_t *slot_table, int layer, const uint16_t *x,

@@ -1,13 +1,10 @@
-"""Host-side checks of the C ABI and of the in-register FP4 decoder (no GPU):
-the libraries load and export every declared symbol, argument checks reject
-bad configs, the slot size matches the page's byte count, and the decoder's
-integer arithmetic (compiled for the host with g++) is exact."""
+"""Host-side checks of the C ABI (no GPU): the libraries load and export
+every declared symbol, argument checks reject bad configs, and the slot size
+matches the page's byte count."""
 import ctypes
 import os
 import re
-import subprocess
 
-import numpy as np
 import pytest
 
 from fp4_routed_expert_router_b200 import build as pkg_build
@@ -75,48 +72,7 @@ def test_null_context_rejected(lib):
     assert lib.moe_fp4_residency_stats(None, None) == moe.EINVAL
     assert lib.moe_fp4_expert_outputs(None, 0, None, 0, None, None, None) == moe.EINVAL
     assert lib.moe_fp4_combine(None, 0, None, None, None, None, None, None) == moe.EINVAL
+    assert lib.moe_fp4_route_forward(None, 0, None, None, None, 0, None, None, None, None, None, None, None,
+                                     None) == moe.EINVAL
+    assert lib.moe_fp4_set_option(None, moe.OPT_WAIT_LIMIT_US, 10) == moe.EINVAL
     lib.moe_fp4_destroy(None)
-
-
-_HARNESS = r"""
-#include "fp4_decode.cuh"
-#include <cstdio>
-#include <cstdint>
-using namespace moe;
-// stdin: lines "scale word"; stdout: the four decoded bf16x2 words
-int main() {
-    unsigned s; unsigned long long v;
-    while (std::scanf("%u %llx", &s, &v) == 2) {
-        uint32_t o[4];
-        fp4_decode8(fp4_reencode_word((uint32_t)v), make_fp4_lut(s), o);
-        std::printf("%08x %08x %08x %08x\n", o[0], o[1], o[2], o[3]);
-    }
-    return 0;
-}
-"""
-
-
-def test_register_decoder_is_exact(tmp_path):
-    """Slot re-encoding + PRMT decode == table value * 2^(s-127), for every
-    supported scale byte and random code words."""
-    src = tmp_path / "h.cpp"
-    exe = tmp_path / "h"
-    src.write_text(_HARNESS)
-    subprocess.check_call(["g++", "-O2", "-std=c++17", "-x", "c++",
-                           "-I", os.path.join(ROOT, "fp4_routed_expert_router_b200", "csrc"),
-                           str(src), "-o", str(exe)])
-    rng = np.random.default_rng(0)
-    scales = np.repeat(np.arange(2, 253), 40)
-    words = rng.integers(0, 2 ** 32, size=scales.size, dtype=np.uint64)
-    words[:16] = np.array([0x76543210, 0xFEDCBA98] * 8, dtype=np.uint64)
-    inp = "".join(f"{s} {w:x}\n" for s, w in zip(scales, words))
-    out = subprocess.run([str(exe)], input=inp, capture_output=True, text=True, check=True).stdout.split()
-    dec = np.array([int(v, 16) for v in out], dtype=np.uint64).reshape(-1, 4)
-    tab = helpers.e2m1_table()
-    for n in range(8):
-        bits = ((dec[:, n // 2] >> np.uint64(16 * (n % 2))) & np.uint64(0xFFFF)).astype(np.uint16)
-        got = helpers.bf16_bits_to_f64(bits)
-        codes = ((words >> np.uint64(4 * n)) & np.uint64(15)).astype(np.int64)
-        want = tab[codes] * np.exp2(scales.astype(np.float64) - 127)
-        assert np.array_equal(got, want)
-        assert np.array_equal(np.signbit(got), np.signbit(want))

@@ -24,13 +24,15 @@ def bench():
 
 
 def test_decode_roofline_is_hbm_with_algorithmic_bytes(bench):
+    """The one-kernel decode step: its algorithmic bytes are the six experts'
+    full objects (w1, w3, w2 codes and scales), 6 x 18,800,640 bytes."""
     from fp4_routed_expert_router_b200 import synth
     wl = synth.WORKLOADS["decode_b1"]
-    r = bench.roofline(wl, {"kernel_ms": {"gemv_up": 0.040, "route": 0.01}, "active": 6.0}, PEAKS, "test")
-    up_bytes = 6 * 2 * (2304 * 5120 // 2 + 2304 * 5120 // 32)
-    assert r["bound"] == "hbm" and r["kernel"] == "gemv_up"
-    assert r["algorithmic_bytes_per_launch"] == up_bytes == 75_202_560
-    assert r["achieved"] == pytest.approx(up_bytes / 40e-6 / 1e9)
+    r = bench.roofline(wl, {"kernel_ms": {"decode_layer": 0.030}, "active": 6.0}, PEAKS, "test")
+    layer_bytes = 6 * (3 * 2304 * 5120 // 2 + 3 * 2304 * 5120 // 32)
+    assert r["bound"] == "hbm" and r["kernel"] == "decode_layer"
+    assert r["algorithmic_bytes_per_launch"] == layer_bytes == 112_803_840
+    assert r["achieved"] == pytest.approx(layer_bytes / 30e-6 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["hbm_gbs"])
 
 
@@ -47,7 +49,7 @@ def test_prefill_roofline_picks_the_bound_by_intensity(bench):
 
 
 def test_stored_traffic_requires_matching_sources(bench, tmp_path):
-    files = ["fp4_decode.cuh", "slot_layout.cuh"]
+    files = ["fp4_cvt.cuh", "slot_layout.cuh"]
     rec = {"k@w": {"bytes_per_launch": 1234, "files": files, "source_digest": bench.source_digest(files)}}
     p = tmp_path / "traffic.json"
     p.write_text(json.dumps(rec))

@@ -54,6 +54,28 @@ def test_tiny_forced_paths(tiny, path, T):
     check_y(y, y_ref)
 
 
+@pytest.mark.parametrize("T", [1, 4, 7])
+def test_tiny_route_forward_one_launch(tiny, T):
+    """moe_fp4_route_forward routes inside the layer kernel (every CTA routes,
+    the first writes the routing): routing bit-exact against the oracle, y
+    within the bar, and identical, bit for bit, to route + forward."""
+    wl = tiny.wl
+    logits, _ = synth.layer_inputs(wl, 0, 3000 + T, tokens=T)
+    x = to_dev(synth.gen_x(wl.seed, T, wl.hidden, 3000 + T))
+    tiny.ctx.set_path(moe.PATH_AUTO)
+    r, y = tiny.ctx.route_forward(0, to_dev(logits), x)
+    torch.cuda.synchronize()
+    rc, msg = tiny.ctx.last_error()
+    assert rc == moe.OK, msg
+    ids, w = check_routing(r, logits, wl.top_k, wl.n_experts)
+    check_y(y.cpu().numpy(), tiny.oracle_y(0, synth.gen_x(wl.seed, T, wl.hidden, 3000 + T), ids, w, range(T)))
+    r2 = tiny.ctx.route(0, to_dev(logits))
+    y2 = tiny.ctx.forward(0, x, r2)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    assert torch.equal(r.weights, r2.weights)
+
+
 def test_tiny_zero_tokens(tiny):
     r = tiny.ctx.alloc_routing(0)
     logits = torch.empty((0, tiny.wl.n_experts), dtype=torch.float32, device="cuda")

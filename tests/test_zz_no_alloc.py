@@ -49,11 +49,20 @@ def test_noalloc_matches_forward_twice(name, T):
         f.close()
 
 
-def test_noalloc_rejects_sizes_beyond_the_scratch():
+def _need(T: int, wl) -> int:
+    """Scratch bytes of a call, as the header states them (each part rounded up to 256)."""
+    H, I, k = wl.hidden, wl.inter, wl.top_k
+    parts = [T * H * 2, T * 4, T * k * I * 2, T * k * (I // 32) * 4, T * k * H * 4]
+    return sum((p + 255) // 256 * 256 for p in parts) + (H // 32) * 4
+
+
+def test_noalloc_rejects_sizes_beyond_the_limits():
     wl = synth.WORKLOADS["decode_b1"]
     cfg = moe.Config(wl.hidden, wl.inter, wl.n_experts, wl.top_k, 1, 1, 4096)
-    per_entry = 2 * wl.inter + 4 * wl.hidden
-    T = (16 << 20) // (per_entry * wl.top_k) + 1        # first T that cannot fit
+    # the largest T whose scratch fits the 16 MiB array
+    T_ok = max(T for T in range(1, 512) if _need(T, wl) <= (16 << 20))
+    assert T_ok == 103
+    T = T_ok + 1
     x = torch.zeros((T, wl.hidden), dtype=torch.int16, device="cuda")
     y = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
     r = moe.Routing(torch.zeros((T, 6), dtype=torch.int32, device="cuda"),
@@ -64,5 +73,9 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     arena = torch.empty(256, dtype=torch.uint8, device="cuda")
     table = torch.full((1, 384), -1, dtype=torch.int32, device="cuda")
     assert moe.forward_noalloc(cfg, arena.data_ptr(), table, 0, x, r, y) == moe.EINVAL
-    assert moe.forward_noalloc(cfg, arena.data_ptr(), table, 0, x[: T - 1], r, y) == moe.OK
+    assert moe.forward_noalloc(cfg, arena.data_ptr(), table, 0, x[:T_ok], r, y) == moe.OK
+    # router weights that are not 4-byte aligned are an argument error, before any launch
+    wbad = r.weights.reshape(-1).view(torch.uint8)[1:]
+    assert moe.forward_noalloc(cfg, arena.data_ptr(), table, 0, x[:1],
+                               moe.Routing(r.ids, wbad, r.counts, r.offsets, r.perm), y) == moe.EINVAL
     torch.cuda.synchronize()
