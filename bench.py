@@ -62,7 +62,7 @@ def workload_config(wl: synth.Workload, graph: bool) -> dict:
         "expert_bytes": wl.expert_bytes, "weights": "fp4 e2m1 + ue8m0 per 32 along K",
         "logits": f"N(0,1) + Zipf(1.1) bias, alpha {wl.zipf_alpha}",
         "scale_exponents": f"uniform {wl.scale_lo}..{wl.scale_hi}",
-        "l2": "flushed between timed steps (2x L2 write)",
+        "l2": "flushed between timed steps (2x L2 write, then its lines discarded)",
         "launch": ("cuda graph of moe_fp4_route_forward" if graph else "eager moe_fp4_route_forward") +
                   (" (one persistent kernel per step)" if wl.tokens * wl.top_k <= 64 else
                    " (route kernel, then the expert kernels)"),
@@ -285,7 +285,7 @@ class Bench:
         def stage(i):
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
             l_buf.copy_(pool_l[i % npool], non_blocking=True)
-            flush.fill_(float(i))
+            moe.l2_flush(flush, float(i), stream)
 
         out = {}
         graph = None
@@ -358,7 +358,7 @@ class Bench:
                 e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                           for _ in range(steps)]
                 for i in range(steps):
-                    flush.fill_(float(i))
+                    moe.l2_flush(flush, float(i), stream)
                     e2e_ev[i][0].record(stream)
                     x_buf.copy_(hx[i % npool], non_blocking=True)
                     l_buf.copy_(hl[i % npool], non_blocking=True)
@@ -427,7 +427,7 @@ def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
         def stage(i):
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
             l_buf.copy_(pool_l[i % npool], non_blocking=True)
-            flush.fill_(float(i))
+            moe.l2_flush(flush, float(i), stream)
 
         graph = None
         with torch.cuda.stream(stream):

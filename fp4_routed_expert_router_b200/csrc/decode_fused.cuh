@@ -83,9 +83,9 @@ struct DecodeArgs {
     uint16_t* xh;                // [T,H] f16 workspace: x * 2^sigma_t (more than one token)
     float* xs;                   // [T]   2^-sigma_t
     uint16_t* hh;                // [T*k, I] f16 workspace (grouped order): h * 2^sigma
-    float* hs;                   // [T*k, I/32] 2^-sigma per (entry, 32-K block)
+    uint8_t* hs;                 // [T*k, I/32] 127 - sigma per (entry, 32-K block): h = hh * 2^(hs-127)
     float* obuf;                 // [T*k, H] fp32 per-entry outputs, entry order t*k+j
-    int* tile_cnt;               // [H/32] combine arrival counters
+    int* tile_cnt;               // [H/16] combine arrival counters
     unsigned int* gbar;          // [4] grid barriers: {count, generation} x 2
     float* y;                    // [T,H] or NULL (per-entry outputs only)
     uint16_t* x_out;             // [T,H] or NULL
@@ -137,18 +137,20 @@ __device__ __forceinline__ void dec_grid_barrier(unsigned int* cnt, unsigned int
     }
 }
 
-// One unit of MMAs: two 16-row A tiles (w1 and w3 rows of one row block, or
-// two row blocks of w2) x 256 (or 128) K against B fragments.  bfrag(q, j)
-// returns this lane's B fragment of 32-K block j of 128-K group q; bscale(q,
-// j, col) the block's activation scale of accumulator column 2c + col (down
-// GEMM; 1 for the up GEMM).  Adds each 32-K block's fp32 result, times
-// 2^(s-127) of its row and the activation scale, into acc[tile*4 ..].  The
-// two MMAs of a block (K 0-15, 16-31) accumulate separately, so they do not
-// wait for each other.
+// One unit of MMAs: two 16-row x 256 (or 128) K A tiles -- w1 and w3 rows
+// of one row block (up), or two consecutive K blocks of the same w2 rows
+// (down; the second may be absent: code1 == NULL) -- against B fragments.
+// bfrag(m, q, j) returns this lane's B fragment for 32-K block j of 128-K
+// group q of tile m; bscale(m, q, j, col) the block's activation scale of
+// accumulator column 2c + col (down GEMM; 1 for the up GEMM).  Adds each
+// 32-K block's fp32 result, times 2^(s-127) of its row and the activation
+// scale, into acc[m*4 ..].  The two MMAs of a block (K 0-15, 16-31)
+// accumulate separately, so they do not wait for each other.
 template <int NTOK, int Q, typename BF, typename BS>
 __device__ __forceinline__ void dec_unit_mma(const uint8_t* code0, const uint8_t* scl0, const uint8_t* code1,
                                              const uint8_t* scl1, int rowbytes, int sb, int g, int c, BF&& bfrag,
                                              BS&& bscale, float (&acc)[8]) {
+    const int ntile = code1 == nullptr ? 1 : 2;
     const int off_g = g * rowbytes, off_g8 = (g + 8) * rowbytes;
     auto group = [&](int q) {
         const int chunk = swizzle_chunk(4 * q + c, g, rowbytes) * 16;   // same for rows g and g + 8
@@ -156,8 +158,8 @@ __device__ __forceinline__ void dec_unit_mma(const uint8_t* code0, const uint8_t
         uint32_t sg[2][2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            const uint8_t* codes = m == 0 ? code0 : code1;
-            const uint8_t* scl = m == 0 ? scl0 : scl1;
+            const uint8_t* codes = (m == 0 || ntile == 1) ? code0 : code1;
+            const uint8_t* scl = (m == 0 || ntile == 1) ? scl0 : scl1;
             A[m][0] = *reinterpret_cast<const uint4*>(codes + off_g + chunk);
             A[m][1] = *reinterpret_cast<const uint4*>(codes + off_g8 + chunk);
             sg[m][0] = *reinterpret_cast<const uint32_t*>(scl + g * sb + 4 * q);
@@ -165,11 +167,12 @@ __device__ __forceinline__ void dec_unit_mma(const uint8_t* code0, const uint8_t
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 xb = bfrag(q, j);
-            const float c0 = bscale(q, j, 0);
-            const float c1 = NTOK > 1 ? bscale(q, j, 1) : 0.0f;
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
+                if (m >= ntile) break;
+                const uint4 xb = bfrag(m, q, j);
+                const float c0 = bscale(m, q, j, 0);
+                const float c1 = NTOK > 1 ? bscale(m, q, j, 1) : 0.0f;
                 const uint4& A0 = A[m][0];
                 const uint4& A1 = A[m][1];
                 uint32_t pa[4], pb[4];
@@ -260,7 +263,8 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
         gen_start[1] = g1;
         fence_barrier_init();
     }
-    for (int e = tid; e < E; e += blockDim.x) slot_s[e] = __ldg(a.slot_table + static_cast<size_t>(a.layer) * E + e);
+    if (warp == NW)   // the producer warp fetches this layer's slot table row while the others route
+        for (int e = lane; e < E; e += 32) slot_s[e] = __ldg(a.slot_table + static_cast<size_t>(a.layer) * E + e);
     // one token: this thread's words of x, fetched now and converted after routing
     constexpr int XW = 8;                              // words of x per consumer thread (H <= 8 * 2 * 448)
     uint32_t xw[XW];
@@ -384,15 +388,16 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
     __syncthreads();
 
     const int n_gs = n_gs_s;
-    const int tiles_up = I / 32, tiles_dn = H / 32;
-    const int upi = 2 * L.nfu, dpi = L.nfd;          // units per item
+    const int tiles_up = I / 32, tiles_dn = H / 16;  // up items: 32 rows of w1/w3; down items: 16 rows of w2
+    const int upi = 2 * L.nfu;                       // units per up item (shared by the CTA's warps)
+    const int dpi = (L.nfd + 1) / 2;                 // units per down item (one warp): two K blocks each
     const int N_up = n_gs * tiles_up, N_dn = n_gs * tiles_dn;
     const int up0 = static_cast<int>((static_cast<long long>(N_up) * b) / G);
     const int up1 = static_cast<int>((static_cast<long long>(N_up) * (b + 1)) / G);
     const int dn0 = static_cast<int>((static_cast<long long>(N_dn) * b) / G);
     const int dn1 = static_cast<int>((static_cast<long long>(N_dn) * (b + 1)) / G);
     const int n_up_units = (up1 - up0) * upi;
-    const int n_units = n_up_units + (dn1 - dn0) * dpi;
+    const int n_dn_items = dn1 - dn0;                // local down item d goes to warp d % NW
     // grouped position -> entry t*k+j (and its token row of x); -1 for an
     // entry outside [0, T*k) (a routing that is not of these tokens)
     auto entry_of = [&](int pos) -> int {
@@ -413,21 +418,17 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
         const uint64_t pol = policy_evict_first();
         const int w = lane;
         const bool serve = w < NW;
-        int i = 0, u = w;
+        int i = 0, u = w;                                   // up: unit u = w + 14 i
         int li = u / upi, r = u - li * upi;                 // up unit: item, unit in item
-        bool down = false;
+        int dl = w, dv = 0;                                 // down: local item dl of this warp, unit dv in it
         bool stop = false;
         uint64_t idle_since = 0;
         for (;;) {
-            const bool more = serve && !stop && u < n_units;
+            const bool down = u >= n_up_units;
+            const bool more = serve && !stop && (down ? dl < n_dn_items : true);
             if (!__any_sync(0xFFFFFFFFu, more)) break;
             bool progress = false;
             if (more) {
-                if (!down && u >= n_up_units) {              // first down unit of this lane
-                    down = true;
-                    li = (u - n_up_units) / dpi;
-                    r = u - n_up_units - li * dpi;
-                }
                 const int ring_i = i % spw;
                 const int sl = w + NW * ring_i;
                 if (i < spw || mbar_test(&empty[sl], ((i / spw) - 1) & 1)) {
@@ -443,26 +444,24 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
                             bulk_g2s(dst, a.arena + static_cast<size_t>(slot) * a.slot_bytes + src,
                                      static_cast<uint32_t>(L.UB), &full[sl], pol);
                         }
+                        u += NW;
                         r += NW;
                         while (r >= upi) { r -= upi; ++li; }
                     } else {
-                        const int gi = dn0 + li, gs = gi / tiles_dn, tile = gi - gs * tiles_dn;
+                        const int gi = dn0 + dl, gs = gi / tiles_dn, tile = gi - gs * tiles_dn;
                         const int slot = act_slot[gs_a[gs]];
+                        const int nb = min(2, L.nfd - 2 * dv);   // K blocks of this unit
                         if (slot < 0) {
                             mbar_arrive(&full[sl]);
                         } else {
-                            const uint8_t* base = a.arena + static_cast<size_t>(slot) * a.slot_bytes + L.up_bytes;
-                            mbar_arrive_expect_tx(&full[sl], static_cast<uint32_t>(2 * L.DB));
-                            bulk_g2s(dst, base + static_cast<size_t>((2 * tile) * L.nfd + r) * L.DB,
-                                     static_cast<uint32_t>(L.DB), &full[sl], pol);
-                            bulk_g2s(dst + L.DB, base + static_cast<size_t>((2 * tile + 1) * L.nfd + r) * L.DB,
-                                     static_cast<uint32_t>(L.DB), &full[sl], pol);
+                            const uint8_t* src = a.arena + static_cast<size_t>(slot) * a.slot_bytes + L.up_bytes +
+                                                 static_cast<size_t>(tile * L.nfd + 2 * dv) * L.DB;
+                            mbar_arrive_expect_tx(&full[sl], static_cast<uint32_t>(nb * L.DB));
+                            bulk_g2s(dst, src, static_cast<uint32_t>(nb * L.DB), &full[sl], pol);
                         }
-                        r += NW;
-                        while (r >= dpi) { r -= dpi; ++li; }
+                        if (++dv == dpi) { dv = 0; dl += NW; }
                     }
                     ++i;
-                    u += NW;
                     progress = true;
                     idle_since = 0;
                 } else if (*abort_flag) {
@@ -472,7 +471,7 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
                     if (idle_since == 0) {
                         idle_since = now;
                     } else if (now - idle_since > a.timeout_ns) {
-                        latch_error(a.err, ERR_ETIMEOUT, u, KID_UP);
+                        latch_error(a.err, ERR_ETIMEOUT, i, KID_UP);
                         *abort_flag = 1;
                         stop = true;
                     }
@@ -625,7 +624,7 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
                 const float hq = __uint_as_float(hb << 16) * pow2i(sg);
                 const uint32_t h16 = f32x2_to_f16x2(hq, 0.0f) & 0xFFFFu;
                 a.hh[static_cast<size_t>(p0 + t) * I + tile * 32 + lane] = static_cast<uint16_t>(h16);
-                if (lane == 0) a.hs[static_cast<size_t>(p0 + t) * (I / 32) + tile] = pow2i(-sg);
+                if (lane == 0) a.hs[static_cast<size_t>(p0 + t) * (I / 32) + tile] = static_cast<uint8_t>(127 - sg);
             }
             if (slot < 0 && lane == 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gsi]], KID_UP);
         };
@@ -665,12 +664,12 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
                 latch_error(a.err, ERR_ETIMEOUT, u, KID_UP);
             if (slot >= 0) {
                 const uint8_t* stg = ring + static_cast<size_t>(sl) * p.unit_bytes;
-                auto bfrag = [&](int q, int j) -> uint4 {
+                auto bfrag = [&](int, int q, int j) -> uint4 {
                     if (NTOK == 1)   // one token: x (or the zero row) in shared memory, read as needed
                         return *reinterpret_cast<const uint4*>(bsrc + 128 * q + 32 * j);
                     return xb[NTOK == 1 ? 0 : q][j];
                 };
-                auto bscale = [](int, int, int) -> float { return 1.0f; };
+                auto bscale = [](int, int, int, int) -> float { return 1.0f; };
                 dec_unit_mma<NTOK, Q>(stg, stg + 32 * rowbytes, stg + 16 * rowbytes, stg + 32 * rowbytes + 16 * sb,
                                       rowbytes, sb, g, c, bfrag, bscale, acc);
             }
@@ -686,71 +685,48 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
 
     // ---------------------------------------------------------------- barrier: h complete
     if (a.y != nullptr && ctid == 0)
-        for (int i = b; i < H / 32; i += G) a.tile_cnt[i] = 0;
+        for (int i2 = b; i2 < H / 16; i2 += G) a.tile_cnt[i2] = 0;
     dec_named_barrier(1, NW * 32);
     if (ctid == 0)
         dec_grid_barrier(a.gbar + 2, a.gbar + 3, gen_start[1], G, a.timeout_ns, a.err, abort_flag, 1);
     dec_named_barrier(1, NW * 32);
 
     // ---------------------------------------------------------------- phase 2: w2 (+ combine)
+    // Warp w takes local down items w, w + 14, ...: (group, 16 rows of w2)
+    // over all of I, in units of two K blocks, accumulated in registers (no
+    // other warp takes part in an item).
     {
         constexpr int Q = QD;
         const int rowbytes = L.KBd / 2, sb = L.KBd / 32;
-        const int n_up_items = up1 - up0;
-        const int expected = min(dpi, NW);
         const int nblk = I / 32;
+        const int kbpb = L.KBd / 32;                      // 32-K scale blocks per K block
         // one token: stage the h rows of this CTA's groups (one entry each) in shared memory
         const int gs_first = dn0 / tiles_dn;
         const int n_stage = (dn1 > dn0) ? (dn1 - 1) / tiles_dn - gs_first + 1 : 0;
-        const bool staged = NTOK == 1;                  // the plan guarantees n_stage <= kDecStageRows
-        if (staged) {
+        if (NTOK == 1) {
             for (int rr = 0; rr < n_stage && rr < kDecStageRows; ++rr) {
                 const int pr = gs_p0[gs_first + rr];
                 const uint4* sh = reinterpret_cast<const uint4*>(a.hh + static_cast<size_t>(pr) * I);
                 uint4* dh = reinterpret_cast<uint4*>(hsm + static_cast<size_t>(rr) * I);
                 for (int q = ctid; q < I / 8; q += NW * 32) dh[q] = __ldcg(sh + q);
                 for (int q = ctid; q < nblk; q += NW * 32)
-                    hsig[rr * nblk + q] = __ldcg(a.hs + static_cast<size_t>(pr) * nblk + q);
+                    hsig[rr * nblk + q] = __uint_as_float(static_cast<uint32_t>(a.hs[static_cast<size_t>(pr) * nblk + q]) << 23);
             }
             dec_named_barrier(1, NW * 32);
         }
-        int cur = -1;
-        float acc[8];
-        int slot = -1, p0 = 0, ng = 0, tile = 0, gsi = 0;
-        const uint16_t* brow = nullptr;
-        const float* hrow0 = nullptr;   // block scales of the columns 2c (and 2c+1)
-        const float* hrow1 = nullptr;
-        auto epi = [&](int bi) {
-            const int rb = lane >> 4, row = lane & 15;
-            const int u_first = n_up_units + cur * dpi;
-            for (int t = 0; t < ng; ++t) {
-                float o = 0.f;
-                for (int r = 0; r < expected; ++r) {
-                    const int w2 = (u_first + r) % NW;
-                    o += part[(static_cast<size_t>(bi) * NW + w2) * PART + (rb * 16 + row) * TP + (TP == 1 ? 0 : t)];
-                }
-                const int ent = entry_of(p0 + t);
-                if (ent >= 0) a.obuf[static_cast<size_t>(ent) * H + tile * 32 + lane] = (slot >= 0) ? o : 0.0f;
-            }
-            if (slot < 0 && lane == 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gsi]], KID_DOWN);
-            if (a.y == nullptr) return;
-            // the CTA that completes the last item of this 32-row output tile
-            // combines it: lane 0's acquire-release add orders the warp's o
-            // stores before it (the warp barrier orders them before lane 0) and
-            // the last arriver's loads after every other arriver's stores
-            __syncwarp();
-            int lastt = 0;
-            if (lane == 0) {
-                unsigned int old;
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                             : "=r"(old) : "l"(a.tile_cnt + tile) : "memory");
-                lastt = (old == static_cast<unsigned int>(n_gs - 1));
-            }
-            lastt = __shfl_sync(0xFFFFFFFFu, lastt, 0);
+        int pend_tile = -1;                 // tile whose combine add is in flight
+        unsigned int pend_old = 0;          // its result (lane 0)
+        // combine of tile pend_tile if this warp's add was the tile's last:
+        // y[t] over the tile's 16 rows for every token, in fixed j order
+        auto combine_pending = [&]() {
+            if (pend_tile < 0) return;
+            const int lastt = __shfl_sync(0xFFFFFFFFu, pend_old == static_cast<unsigned int>(n_gs - 1) ? 1 : 0, 0);
+            const int tile = pend_tile;
+            pend_tile = -1;
             if (!lastt) return;
             __syncwarp();   // lane 0's acquire before every lane's loads
-            const int n0 = tile * 32 + lane;
-            for (int t = 0; t < a.T; ++t) {
+            const int n0 = tile * 16 + (lane & 15);
+            for (int t = lane >> 4; t < a.T; t += 2) {
                 float yv = 0.f;
                 for (int j = 0; j < k; ++j) {
                     const float wj = routed ? r_w[t * k + j] : __ldg(a.weights + t * k + j);
@@ -763,80 +739,109 @@ moe_fp4_decode_layer(DecodeArgs a, SlotLayout L, DecodePlan p) {
                 }
             }
         };
-        const int u_start = n_up_units + ((warp - n_up_units % NW + NW) % NW);
-        int i = (u_start - warp) / NW;
+        int i = (n_up_units - warp + NW - 1) / NW;       // this warp's up units: its ring position now
+        if (i < 0) i = 0;
         int ring_i = i % spw, par = (i / spw) & 1;
-        int li = (u_start - n_up_units) / dpi, f = u_start - n_up_units - li * dpi;
-        for (int u = u_start; u < n_units; u += NW) {
-            if (li != cur) {
-                if (cur >= 0) flush(n_up_items + cur, acc, expected, epi);
-                cur = li;
+        for (int dl = warp; dl < n_dn_items; dl += NW) {
+            const int gi = dn0 + dl;
+            const int gsi = gi / tiles_dn, tile = gi - gsi * tiles_dn;
+            const int slot = act_slot[gs_a[gsi]];
+            const int p0 = gs_p0[gsi], ng = gs_n[gsi];
+            const uint16_t* brow;
+            const float* hrow0 = nullptr;       // one token: block scales of the entry (shared memory)
+            const uint8_t* hr0 = nullptr;       // block scale exponents of column 2c
+            const uint8_t* hr1 = nullptr;       // and of column 2c + 1
+            if (NTOK == 1) {
+                brow = (g < ng) ? hsm + static_cast<size_t>(gsi - gs_first) * I : zrow;
+                hrow0 = hsig + (gsi - gs_first) * nblk;
+            } else {
+                brow = (g < ng) ? a.hh + static_cast<size_t>(p0 + g) * I : nullptr;
+                hr0 = (2 * c < ng) ? a.hs + static_cast<size_t>(p0 + 2 * c) * nblk : nullptr;
+                hr1 = (2 * c + 1 < ng) ? a.hs + static_cast<size_t>(p0 + 2 * c + 1) * nblk : nullptr;
+            }
+            float acc[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-                const int gi = dn0 + li;
-                gsi = gi / tiles_dn;
-                tile = gi - gsi * tiles_dn;
-                slot = act_slot[gs_a[gsi]];
-                p0 = gs_p0[gsi];
-                ng = gs_n[gsi];
-                if (NTOK == 1) {
-                    brow = (g < ng) ? hsm + static_cast<size_t>(gsi - gs_first) * I : zrow;
-                    hrow0 = hsig + (gsi - gs_first) * nblk;
-                    hrow1 = nullptr;
-                } else {
-                    brow = (g < ng) ? a.hh + static_cast<size_t>(p0 + g) * I : nullptr;
-                    hrow0 = (2 * c < ng || NTOK == 1) ? a.hs + static_cast<size_t>(p0 + (NTOK == 1 ? 0 : 2 * c)) * nblk
-                                                      : nullptr;
-                    hrow1 = (NTOK > 1 && 2 * c + 1 < ng) ? a.hs + static_cast<size_t>(p0 + 2 * c + 1) * nblk : nullptr;
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+            for (int dv = 0; dv < dpi; ++dv) {
+                const int sl = warp + NW * ring_i;
+                const bool two = 2 * dv + 1 < L.nfd;     // second K block present
+                const int kbase = 2 * dv * L.KBd;         // K of this unit's first block
+                uint4 xb[NTOK == 1 ? 1 : 2][NTOK == 1 ? 1 : Q][4];
+                uint32_t hw0[NTOK == 1 ? 1 : 2][NTOK == 1 ? 1 : Q], hw1[NTOK == 1 ? 1 : 2][NTOK == 1 ? 1 : Q];
+                if (NTOK > 1) {   // prefetch B and its block scales (L2) before waiting for the weights
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int q = 0; q < Q; ++q) {
+                            const int kk = kbase + m * L.KBd + 128 * q;
+                            const bool ok = m == 0 || two;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                xb[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q][j] =
+                                    (brow == nullptr || !ok) ? make_uint4(0u, 0u, 0u, 0u)
+                                                             : __ldcg(reinterpret_cast<const uint4*>(brow + kk + 32 * j + 8 * c));
+                            const int kb = kk / 32;   // a multiple of 4 (I/32 too): four exponents in one word
+                            hw0[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q] =
+                                (hr0 == nullptr || !ok) ? 0u : __ldcg(reinterpret_cast<const unsigned int*>(hr0 + kb));
+                            hw1[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q] =
+                                (hr1 == nullptr || !ok) ? 0u : __ldcg(reinterpret_cast<const unsigned int*>(hr1 + kb));
+                        }
                 }
-            }
-            const int sl = warp + NW * ring_i;
-            const uint16_t* bsrc = NTOK == 1 ? brow + (brow == zrow ? 0 : f * L.KBd) + 8 * c
-                                             : (brow == nullptr ? nullptr : brow + f * L.KBd + 8 * c);
-            const int kb0 = f * (L.KBd / 32);
-            uint4 xb[NTOK == 1 ? 1 : Q][4];
-            float hm0[NTOK == 1 ? 1 : Q * 4], hm1[NTOK == 1 ? 1 : Q * 4];
-            if (NTOK > 1) {   // prefetch B and its block scales (L2) before waiting for the weights
-#pragma unroll
-                for (int q = 0; q < Q; ++q) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        xb[NTOK == 1 ? 0 : q][j] = bsrc == nullptr ? make_uint4(0u, 0u, 0u, 0u)
-                                                                   : __ldcg(reinterpret_cast<const uint4*>(bsrc + 128 * q + 32 * j));
-                    const float4 s0 = hrow0 == nullptr ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                                       : __ldcg(reinterpret_cast<const float4*>(hrow0 + kb0 + 4 * q));
-                    const float4 s1 = hrow1 == nullptr ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                                       : __ldcg(reinterpret_cast<const float4*>(hrow1 + kb0 + 4 * q));
-                    hm0[NTOK == 1 ? 0 : 4 * q + 0] = s0.x; hm0[NTOK == 1 ? 0 : 4 * q + 1] = s0.y;
-                    hm0[NTOK == 1 ? 0 : 4 * q + 2] = s0.z; hm0[NTOK == 1 ? 0 : 4 * q + 3] = s0.w;
-                    hm1[NTOK == 1 ? 0 : 4 * q + 0] = s1.x; hm1[NTOK == 1 ? 0 : 4 * q + 1] = s1.y;
-                    hm1[NTOK == 1 ? 0 : 4 * q + 2] = s1.z; hm1[NTOK == 1 ? 0 : 4 * q + 3] = s1.w;
+                if (!mbar_wait(&full[sl], par, abort_flag, a.timeout_ns) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, dl, KID_DOWN);
+                if (slot >= 0) {
+                    const uint8_t* stg = ring + static_cast<size_t>(sl) * p.unit_bytes;
+                    const uint16_t* bsrc = NTOK == 1 ? brow + (brow == zrow ? 0 : kbase) + 8 * c : nullptr;
+                    auto bfrag = [&](int m, int q, int j) -> uint4 {
+                        if (NTOK == 1)   // one token: staged h row (or the zero row) in shared memory
+                            return *reinterpret_cast<const uint4*>(bsrc + (brow == zrow ? 0 : m * L.KBd) + 128 * q +
+                                                                   32 * j);
+                        return xb[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q][j];
+                    };
+                    auto bscale = [&](int m, int q, int j, int col) -> float {
+                        if (NTOK == 1) return hrow0[kbase / 32 + m * kbpb + 4 * q + j];
+                        return ue8m0_mult(col == 0 ? hw0[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q]
+                                                   : hw1[NTOK == 1 ? 0 : m][NTOK == 1 ? 0 : q], j);
+                    };
+                    dec_unit_mma<NTOK, Q>(stg, stg + 16 * rowbytes, two ? stg + L.DB : nullptr,
+                                          two ? stg + L.DB + 16 * rowbytes : nullptr, rowbytes, sb, g, c, bfrag,
+                                          bscale, acc);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[sl]);
+                if (a.y != nullptr) combine_pending();
+                ++i;
+                if (++ring_i == spw) { ring_i = 0; par ^= 1; }
             }
-            if (!mbar_wait(&full[sl], par, abort_flag, a.timeout_ns) && lane == 0)
-                latch_error(a.err, ERR_ETIMEOUT, u, KID_DOWN);
-            if (slot >= 0) {
-                const uint8_t* stg = ring + static_cast<size_t>(sl) * p.unit_bytes;
-                auto bfrag = [&](int q, int j) -> uint4 {
-                    if (NTOK == 1)   // one token: staged h row (or the zero row) in shared memory
-                        return *reinterpret_cast<const uint4*>(bsrc + 128 * q + 32 * j);
-                    return xb[NTOK == 1 ? 0 : q][j];
-                };
-                auto bscale = [&](int q, int j, int col) -> float {
-                    if (NTOK == 1) return hrow0[kb0 + 4 * q + j];
-                    return col == 0 ? hm0[NTOK == 1 ? 0 : 4 * q + j] : hm1[NTOK == 1 ? 0 : 4 * q + j];
-                };
-                dec_unit_mma<NTOK, Q>(stg, stg + 16 * rowbytes, stg + L.DB, stg + L.DB + 16 * rowbytes, rowbytes, sb,
-                                      g, c, bfrag, bscale, acc);
+            // epilogue of the item: o rows of the entries (rows g, g+8 of the tile; columns 2c, 2c+1)
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int col = 2 * c + cc;
+                if (col >= ng || (NTOK == 1 && cc == 1)) continue;
+                const int ent = entry_of(p0 + col);
+                if (ent < 0) continue;
+                float* orow = a.obuf + static_cast<size_t>(ent) * H + tile * 16;
+                orow[g] = slot >= 0 ? acc[cc] + acc[4 + cc] : 0.0f;
+                orow[g + 8] = slot >= 0 ? acc[2 + cc] + acc[6 + cc] : 0.0f;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[sl]);
-            ++i;
-            if (++ring_i == spw) { ring_i = 0; par ^= 1; }
-            f += NW;
-            while (f >= dpi) { f -= dpi; ++li; }
+            if (slot < 0 && lane == 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gsi]], KID_DOWN);
+            if (a.y != nullptr) {
+                // lane 0's acquire-release add orders the warp's o stores before it
+                // (the warp barrier orders them before lane 0) and the last arriver's
+                // loads after every other arriver's stores; its result is looked at
+                // after the warp's next unit (combine_pending)
+                if (pend_tile >= 0) combine_pending();
+                __syncwarp();
+                if (lane == 0) {
+                    unsigned int old;
+                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                                 : "=r"(old) : "l"(a.tile_cnt + tile) : "memory");
+                    pend_old = old;
+                }
+                pend_tile = tile;
+            }
         }
-        if (cur >= 0) flush(n_up_items + cur, acc, expected, epi);
+        if (a.y != nullptr) combine_pending();
     }
 }
 

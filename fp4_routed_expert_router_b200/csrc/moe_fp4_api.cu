@@ -37,11 +37,11 @@ struct moe_fp4_ctx {
     uint16_t* d_xh = nullptr;          // [max_tokens*k, H] f16 prescaled x rows (decode kernel)
     float* d_xs = nullptr;             // [max_tokens*k] their 2^-sigma
     uint16_t* d_hh = nullptr;          // [max_tokens*k, I] f16 prescaled h rows
-    float* d_hs = nullptr;             // [max_tokens*k, I/32] 2^-sigma per (entry, 32-K block)
+    uint8_t* d_hs = nullptr;           // [max_tokens*k, I/32] 127 - sigma per (entry, 32-K block)
     float* d_o = nullptr;              // [max_tokens*k, H] fp32
     float* d_norm = nullptr;           // [max_tokens*k] fp32 (saliency)
     int32_t* d_grp = nullptr;          // expert_outputs grouping: counts [E], offsets [E+1], perm [max_tokens*k]
-    int* d_tile = nullptr;             // [H/32] combine counters of the decode kernel
+    int* d_tile = nullptr;             // [H/16] combine counters of the decode kernel
     unsigned int* d_gbar = nullptr;    // [4] grid barriers of the decode kernel
     int* d_err = nullptr;              // error word [4]
     unsigned int* d_ticket = nullptr;  // route kernel ticket
@@ -365,11 +365,11 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaMalloc(&c->d_xh, sizeof(uint16_t) * ent * H) != cudaSuccess ||
         cudaMalloc(&c->d_xs, sizeof(float) * ent) != cudaSuccess ||
         cudaMalloc(&c->d_hh, sizeof(uint16_t) * ent * I) != cudaSuccess ||
-        cudaMalloc(&c->d_hs, sizeof(float) * ent * (I / 32)) != cudaSuccess ||
+        cudaMalloc(&c->d_hs, ent * (I / 32)) != cudaSuccess ||
         cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
         cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
         cudaMalloc(&c->d_grp, sizeof(int32_t) * (2 * static_cast<size_t>(cfg->n_experts) + 1 + ent)) != cudaSuccess ||
-        cudaMalloc(&c->d_tile, sizeof(int) * (H / 32)) != cudaSuccess ||
+        cudaMalloc(&c->d_tile, sizeof(int) * (H / 16)) != cudaSuccess ||
         cudaMalloc(&c->d_gbar, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
@@ -387,7 +387,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_rowref, 0, rowref_bytes) != cudaSuccess ||
-        cudaMemset(c->d_tile, 0, sizeof(int) * (H / 32)) != cudaSuccess ||
+        cudaMemset(c->d_tile, 0, sizeof(int) * (H / 16)) != cudaSuccess ||
         cudaMemset(c->d_gbar, 0, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
         cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
@@ -901,7 +901,7 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
     // per-entry outputs, combine counters
     const size_t o_xh = 0, o_xs = align256(o_xh + T * H * 2), o_hh = align256(o_xs + T * 4);
     const size_t o_hs = align256(o_hh + ent * I * 2), o_o = align256(o_hs + ent * (I / 32) * 4);
-    const size_t o_tc = align256(o_o + ent * H * 4), need = o_tc + (H / 32) * 4;
+    const size_t o_tc = align256(o_o + ent * H * 4), need = o_tc + (H / 16) * 4;
     if (need > kNoallocScratchBytes) return MOE_FP4_EINVAL;
     const SlotLayout L = make_slot_layout(cfg->hidden, cfg->inter);
     int dev = 0;
@@ -928,7 +928,7 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
     a.xh = reinterpret_cast<uint16_t*>(sp + o_xh);
     a.xs = reinterpret_cast<float*>(sp + o_xs);
     a.hh = reinterpret_cast<uint16_t*>(sp + o_hh);
-    a.hs = reinterpret_cast<float*>(sp + o_hs);
+    a.hs = sp + o_hs;
     a.obuf = reinterpret_cast<float*>(sp + o_o);
     a.tile_cnt = reinterpret_cast<int*>(sp + o_tc);
     a.gbar = d.gbar;

@@ -134,7 +134,11 @@ def l2_flush(buf: torch.Tensor, value: float = 0.0, stream=None) -> None:
     """Push every earlier line out of L2 by writing ``buf`` (larger than L2),
     then drop ``buf``'s own lines without write-back: the next kernel starts
     with a cold, clean L2."""
-    buf.fill_(value)
+    if stream is None:
+        buf.fill_(value)
+    else:
+        with torch.cuda.stream(stream):
+            buf.fill_(value)
     n = buf.numel() * buf.element_size() // 128 * 128
     rc = load_synth().moe_synth_l2_discard(_ptr(buf), n, _stream(stream))
     if rc != 0:

@@ -335,7 +335,7 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
  * library-owned, file-scope device array of 16 MiB (16,777,216 bytes) that
  * every GPU which loads the library holds until the process exits, next to
  * 16 bytes of grid-barrier state.  The scratch must hold
- *   T*H*2 + T*4 + T*k*I*2 + T*k*(I/32)*4 + T*k*H*4 + (H/32)*4 bytes
+ *   T*H*2 + T*4 + T*k*I*2 + T*k*(I/32)*4 + T*k*H*4 + (H/16)*4 bytes
  * (each part rounded up to 256); a larger T, or a shape the decode kernel
  * does not take, returns EINVAL before any launch.  For the V4.1 shape (k = 6)
  * that allows T <= 103.  Up to 16 tokens the combine runs inside the kernel,

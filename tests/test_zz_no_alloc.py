@@ -53,7 +53,7 @@ def _need(T: int, wl) -> int:
     """Scratch bytes of a call, as the header states them (each part rounded up to 256)."""
     H, I, k = wl.hidden, wl.inter, wl.top_k
     parts = [T * H * 2, T * 4, T * k * I * 2, T * k * (I // 32) * 4, T * k * H * 4]
-    return sum((p + 255) // 256 * 256 for p in parts) + (H // 32) * 4
+    return sum((p + 255) // 256 * 256 for p in parts) + (H // 16) * 4
 
 
 def test_noalloc_rejects_sizes_beyond_the_limits():
