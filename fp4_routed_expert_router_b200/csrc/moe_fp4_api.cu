@@ -15,7 +15,7 @@
 #include "../../include/moe_fp4.h"
 #include "common.cuh"
 #include "decode_common.cuh"
-#include "decode_fused.cuh"
+#include "decode_mx.cuh"
 #include "router.cuh"
 #include "slot_layout.cuh"
 #include "residency.h"
@@ -34,15 +34,14 @@ struct moe_fp4_ctx {
     int32_t* d_table = nullptr;        // [L][E]
     uint8_t* d_rowref = nullptr;       // [n_slots][2I + H] largest scale byte of each weight row
     uint8_t* d_staging = nullptr;      // one expert, checkpoint layout
-    uint16_t* d_xh = nullptr;          // [max_tokens*k, H] f16 prescaled x rows (decode kernel)
-    float* d_xs = nullptr;             // [max_tokens*k] their 2^-sigma
-    uint16_t* d_hh = nullptr;          // [max_tokens*k, I] f16 prescaled h rows
-    uint8_t* d_hs = nullptr;           // [max_tokens*k, I/32] 127 - sigma per (entry, 32-K block)
+    uint16_t* d_hh = nullptr;          // [max_tokens*k, I] f16 prescaled h rows (tcgen05 f16 path)
     float* d_o = nullptr;              // [max_tokens*k, H] fp32
     float* d_norm = nullptr;           // [max_tokens*k] fp32 (saliency)
     int32_t* d_grp = nullptr;          // expert_outputs grouping: counts [E], offsets [E+1], perm [max_tokens*k]
-    int* d_tile = nullptr;             // [H/16] combine counters of the decode kernel
-    unsigned int* d_gbar = nullptr;    // [4] grid barriers of the decode kernel
+    // decode kernel (decode_mx.cuh) workspace, for up to mx_ent token-expert entries
+    int mx_ent = 0;
+    uint8_t* d_mx = nullptr;           // one allocation holding the buffers below
+    MxArgs mx{};                       // its buffer pointers (xp, xsf, hp, hsf, part, seq, cnt, ready, zero)
     int* d_err = nullptr;              // error word [4]
     unsigned int* d_ticket = nullptr;  // route kernel ticket
     unsigned long long timeout_ns = 1000000000ull;   // bounded device waits
@@ -145,11 +144,11 @@ cudaError_t launch_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim
 
 // Re-lay one expert from the staging buffer (checkpoint layout: w1, w3, w2
 // codes, then s1, s3, s2 scales, row-major) into its slot (slot_layout.cuh):
-// one thread per 16-byte chunk of codes (four words gathered from the row's
-// 64-byte group, placed in its block at its swizzled position), one per scale
-// byte (checked against the supported range [2, 252]), and one per weight row
-// for the row's largest scale byte (rowref, used by the tcgen05 path).
-// Thread 0 maps (layer, expert) -> slot.
+// one thread per 16-byte chunk of codes (32 codes of one row and one scale
+// block, contiguous in both layouts), one per scale byte (checked against the
+// supported range [2, 252]), and one per weight row for the row's largest
+// scale byte (rowref, used by the f16 tcgen05 path).  Thread 0 maps (layer,
+// expert) -> slot.
 __global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, SlotLayout L,
                                  uint8_t* __restrict__ rowref, int32_t* table, int map_index, int slot, int* err) {
     const size_t H = L.H, I = L.I;
@@ -161,11 +160,11 @@ __global__ void load_slot_kernel(const uint8_t* __restrict__ src, uint8_t* __res
     if (i < 2 * n13 + n2) {
         size_t so, dofs;
         slot_code_chunk(L, i, &so, &dofs);
-        uint4 w;
+        uint4 w;   // the staging buffer is only 4-byte aligned
         w.x = *reinterpret_cast<const uint32_t*>(src + so + 0);
-        w.y = *reinterpret_cast<const uint32_t*>(src + so + 16);
-        w.z = *reinterpret_cast<const uint32_t*>(src + so + 32);
-        w.w = *reinterpret_cast<const uint32_t*>(src + so + 48);
+        w.y = *reinterpret_cast<const uint32_t*>(src + so + 4);
+        w.z = *reinterpret_cast<const uint32_t*>(src + so + 8);
+        w.w = *reinterpret_cast<const uint32_t*>(src + so + 12);
         *reinterpret_cast<uint4*>(dst + dofs) = w;
         return;
     }
@@ -204,57 +203,65 @@ const char* kernel_name(int kid) {
     }
 }
 
-// ---- decode path: the persistent fused layer kernel (decode_fused.cuh)
-// Instantiated for NTOK in {1, 8} (a batch of one token keeps one partial
-// column) and K blocks of 128 or 256 for w1/w3 (QU) and w2 (QD).
-template <int NTOK, int QU, int QD>
-cudaError_t launch_decode_t(const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid,
-                            cudaStream_t s) {
+// ---- decode path: the persistent layer kernel (decode_mx.cuh), one CTA per
+// SM, all co-resident (cooperative launch): CTAs wait on one another's flags.
+cudaError_t launch_mx(const MxArgs& a, const SlotLayout& L, const MxPlan& p, int grid, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kDecThreads);
+    cfg.blockDim = dim3(kMxThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(p.smem_bytes);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs co-resident: the kernel has grid barriers
+    attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe_fp4_decode_layer<NTOK, QU, QD>, a, L, p);
+    return cudaLaunchKernelEx(&cfg, moe_fp4_decode_mx, a, L, p);
 }
 
-template <int NTOK, int QU, int QD>
-cudaError_t allow_decode_smem(int bytes) {
-    return cudaFuncSetAttribute(reinterpret_cast<const void*>(moe_fp4_decode_layer<NTOK, QU, QD>),
+cudaError_t allow_mx_smem(int bytes) {
+    return cudaFuncSetAttribute(reinterpret_cast<const void*>(moe_fp4_decode_mx),
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-cudaError_t allow_decode_smem_all(int bytes) {
-    cudaError_t e = cudaSuccess, r;
-    if ((r = allow_decode_smem<1, 1, 1>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<1, 1, 2>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<1, 2, 1>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<1, 2, 2>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<8, 1, 1>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<8, 1, 2>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<8, 2, 1>(bytes)) != cudaSuccess) e = r;
-    if ((r = allow_decode_smem<8, 2, 2>(bytes)) != cudaSuccess) e = r;
-    return e;
+// Byte offsets of the decode workspace buffers inside one allocation (each
+// 256-byte aligned): first the part that persists across launches at fixed
+// offsets -- the launch sequence number, 1 KB of zeros, the up-item flags and
+// the tagged counters (all zero at creation) -- then the per-launch buffers.
+struct MxOffsets {
+    size_t seq, zero, ready, cnt, xp, xsf, hp, hsf, part, total;
+};
+inline MxOffsets mx_offsets(const MxSizes& z, size_t ready_bytes, size_t cnt_bytes) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    MxOffsets o;
+    o.seq = 0;
+    o.zero = 256;
+    o.ready = 256 + 1024;
+    o.cnt = up(o.ready + ready_bytes);
+    o.xp = up(o.cnt + 2 * cnt_bytes);   // two counter banks
+    o.xsf = up(o.xp + z.xp);
+    o.hp = up(o.xsf + z.xsf);
+    o.hsf = up(o.hp + z.hp);
+    o.part = up(o.hsf + z.hsf);
+    o.total = up(o.part + z.part);
+    return o;
 }
-
-cudaError_t launch_decode(const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid, cudaStream_t s) {
-    const bool qu = L.KBu == 256, qd = L.KBd == 256;
-    if (p.tp == 1) {
-        if (qu) return qd ? launch_decode_t<1, 2, 2>(a, L, p, grid, s) : launch_decode_t<1, 2, 1>(a, L, p, grid, s);
-        return qd ? launch_decode_t<1, 1, 2>(a, L, p, grid, s) : launch_decode_t<1, 1, 1>(a, L, p, grid, s);
-    }
-    if (qu) return qd ? launch_decode_t<8, 2, 2>(a, L, p, grid, s) : launch_decode_t<8, 2, 1>(a, L, p, grid, s);
-    return qd ? launch_decode_t<8, 1, 2>(a, L, p, grid, s) : launch_decode_t<8, 1, 1>(a, L, p, grid, s);
+inline void mx_bind(MxArgs* a, uint8_t* base, const MxOffsets& o, size_t cnt_bytes) {
+    a->seq = reinterpret_cast<unsigned int*>(base + o.seq);
+    a->cnt = reinterpret_cast<unsigned int*>(base + o.cnt);
+    a->cnt_cap = static_cast<int>(cnt_bytes / sizeof(unsigned int));
+    a->ready = reinterpret_cast<unsigned int*>(base + o.ready);
+    a->zero = base + o.zero;
+    a->xp = base + o.xp;
+    a->xsf = base + o.xsf;
+    a->hp = base + o.hp;
+    a->hsf = base + o.hsf;
+    a->part = reinterpret_cast<float*>(base + o.part);
 }
 
 // Launch the decode kernel bracketed by profiling events when the context
 // profiles (c may be NULL).
-cudaError_t decode_run(moe_fp4_ctx* c, const DecodeArgs& a, const SlotLayout& L, const DecodePlan& p, int grid,
+cudaError_t decode_run(moe_fp4_ctx* c, const MxArgs& a, const SlotLayout& L, const MxPlan& p, int grid,
                        cudaStream_t s) {
     const bool prof = c && c->profile && c->prof.size() < 65536;
     cudaEvent_t ea = nullptr, eb = nullptr;
@@ -263,7 +270,7 @@ cudaError_t decode_run(moe_fp4_ctx* c, const DecodeArgs& a, const SlotLayout& L,
         eb = take_event(c);
         cudaEventRecord(ea, s);
     }
-    cudaError_t e = launch_decode(a, L, p, grid, s);
+    cudaError_t e = launch_mx(a, L, p, grid, s);
     if (prof) {
         cudaEventRecord(eb, s);
         c->prof.push_back({"decode_layer", ea, eb});
@@ -271,9 +278,15 @@ cudaError_t decode_run(moe_fp4_ctx* c, const DecodeArgs& a, const SlotLayout& L,
     return e;
 }
 
+// Plan of a decode launch over the context's workspace (ok = 0 if it does not fit).
+MxPlan decode_plan(moe_fp4_ctx* c, int T, int k, bool routed) {
+    if (T * k > c->mx_ent || T > c->mx_ent) return MxPlan{};
+    return make_mx_plan(c->lay, T, k, c->cfg.n_experts, routed, c->smem_optin);
+}
+
 // Decode arguments over the context's workspace.
-DecodeArgs decode_args(moe_fp4_ctx* c, int layer, int k, int T, const uint16_t* x) {
-    DecodeArgs a{};
+MxArgs decode_args(moe_fp4_ctx* c, int layer, int k, int T, const uint16_t* x) {
+    MxArgs a = c->mx;
     a.arena = c->arena;
     a.slot_bytes = c->slot_bytes;
     a.slot_table = c->d_table;
@@ -284,13 +297,7 @@ DecodeArgs decode_args(moe_fp4_ctx* c, int layer, int k, int T, const uint16_t* 
     a.I = c->cfg.inter;
     a.T = T;
     a.x = x;
-    a.xh = c->d_xh;
-    a.xs = c->d_xs;
-    a.hh = c->d_hh;
-    a.hs = c->d_hs;
     a.obuf = c->d_o;
-    a.tile_cnt = c->d_tile;
-    a.gbar = c->d_gbar;
     a.err = c->d_err;
     a.timeout_ns = c->timeout_ns;
     return a;
@@ -362,22 +369,27 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     if (cudaMalloc(&c->d_table, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMalloc(&c->d_rowref, rowref_bytes) != cudaSuccess ||
         cudaMalloc(&c->d_staging, c->slot_bytes) != cudaSuccess ||
-        cudaMalloc(&c->d_xh, sizeof(uint16_t) * ent * H) != cudaSuccess ||
-        cudaMalloc(&c->d_xs, sizeof(float) * ent) != cudaSuccess ||
         cudaMalloc(&c->d_hh, sizeof(uint16_t) * ent * I) != cudaSuccess ||
-        cudaMalloc(&c->d_hs, ent * (I / 32)) != cudaSuccess ||
         cudaMalloc(&c->d_o, sizeof(float) * ent * H) != cudaSuccess ||
         cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
         cudaMalloc(&c->d_grp, sizeof(int32_t) * (2 * static_cast<size_t>(cfg->n_experts) + 1 + ent)) != cudaSuccess ||
-        cudaMalloc(&c->d_tile, sizeof(int) * (H / 16)) != cudaSuccess ||
-        cudaMalloc(&c->d_gbar, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
         cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
         cudaGetLastError();
         return bail(MOE_FP4_ENOMEM);
     }
     c->smem_optin -= 1024;   // room for the kernels' static shared memory
-    if (allow_decode_smem_all(c->smem_optin) != cudaSuccess) {
+    // decode workspace: batches up to kMxMaxEntries token-expert entries
+    c->mx_ent = static_cast<int>(ent < static_cast<size_t>(kMxMaxEntries) ? ent : kMxMaxEntries);
+    const MxSizes mz = mx_sizes(c->lay, c->mx_ent, 1, cfg->n_experts, c->sm_count);
+    const MxOffsets mo = mx_offsets(mz, mz.ready, mz.cnt);
+    if (cudaMalloc(&c->d_mx, mo.total) != cudaSuccess) {
+        cudaGetLastError();
+        return bail(MOE_FP4_ENOMEM);
+    }
+    mx_bind(&c->mx, c->d_mx, mo, mz.cnt);
+    if (allow_mx_smem(c->smem_optin) != cudaSuccess ||
+        cudaMemset(c->d_mx, 0, mo.xp) != cudaSuccess) {   // sequence, counters, flags, zero block
         cudaGetLastError();
         return bail(MOE_FP4_ECUDA);
     }
@@ -387,8 +399,6 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     }
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_rowref, 0, rowref_bytes) != cudaSuccess ||
-        cudaMemset(c->d_tile, 0, sizeof(int) * (H / 16)) != cudaSuccess ||
-        cudaMemset(c->d_gbar, 0, sizeof(unsigned int) * 4) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
         cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
@@ -407,15 +417,11 @@ void moe_fp4_destroy(moe_fp4_ctx* c) {
     cudaFree(c->d_table);
     cudaFree(c->d_rowref);
     cudaFree(c->d_staging);
-    cudaFree(c->d_xh);
-    cudaFree(c->d_xs);
     cudaFree(c->d_hh);
-    cudaFree(c->d_hs);
     cudaFree(c->d_o);
     cudaFree(c->d_norm);
     cudaFree(c->d_grp);
-    cudaFree(c->d_tile);
-    cudaFree(c->d_gbar);
+    cudaFree(c->d_mx);
     for (int b = 0; b < 2; ++b) {
         if (c->d_stage2[b]) cudaFree(c->d_stage2[b]);
         if (c->st_ready[b]) cudaEventDestroy(c->st_ready[b]);
@@ -625,13 +631,13 @@ moe_fp4_status moe_fp4_forward(moe_fp4_ctx* c, int layer, const uint16_t* x, int
     const int H = g.hidden, I = g.inter, E = g.n_experts, k = g.top_k;
     const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
     if (!want_tc) {   // decode path: one persistent kernel (+ the combine for batches above 16 tokens)
-        const DecodePlan p = make_decode_plan(c->lay, T, k, E, false, c->smem_optin, c->sm_count);
+        const MxPlan p = decode_plan(c, T, k, false);
         if (p.ok) {
-            DecodeArgs a = decode_args(c, layer, k, T, x);
+            MxArgs a = decode_args(c, layer, k, T, x);
             a.weights = const_cast<float*>(weights);
             a.offsets = const_cast<int32_t*>(offsets);
             a.perm = const_cast<int32_t*>(perm);
-            const bool fuse = T <= kDecCombineMax;
+            const bool fuse = T <= kMxCombineMax;
             a.y = fuse ? y : nullptr;
             a.x_out = fuse ? x_out : nullptr;
             cudaError_t e = decode_run(c, a, c->lay, p, c->sm_count, s);
@@ -671,9 +677,9 @@ moe_fp4_status moe_fp4_route_forward(moe_fp4_ctx* c, int layer, const float* log
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && tc_prefers(T, g));
     if (T > 0 && !want_tc) {
-        const DecodePlan p = make_decode_plan(c->lay, T, g.top_k, g.n_experts, true, c->smem_optin, c->sm_count);
+        const MxPlan p = decode_plan(c, T, g.top_k, true);
         if (p.ok) {   // routing inside the layer kernel: one launch for the whole layer
-            DecodeArgs a = decode_args(c, layer, g.top_k, T, x);
+            MxArgs a = decode_args(c, layer, g.top_k, T, x);
             a.logits = logits;
             a.keep = keep_mask;
             a.ids = ids;
@@ -715,9 +721,9 @@ moe_fp4_status moe_fp4_expert_outputs(moe_fp4_ctx* c, int layer, const uint16_t*
     if (e != cudaSuccess) return cuda_fail(c, e, "expert_outputs: group launch");
     const bool want_tc = (c->path == MOE_FP4_PATH_TC) || (c->path == MOE_FP4_PATH_AUTO && 4LL * n >= 3LL * E);
     if (!want_tc) {
-        const DecodePlan p = make_decode_plan(c->lay, n, 1, E, false, c->smem_optin, c->sm_count);
+        const MxPlan p = decode_plan(c, n, 1, false);
         if (p.ok) {   // every row its own token (k = 1), per-entry outputs only
-            DecodeArgs a = decode_args(c, layer, 1, n, x);
+            MxArgs a = decode_args(c, layer, 1, n, x);
             a.offsets = offsets;
             a.perm = perm;
             a.obuf = o;
@@ -830,23 +836,22 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx* c, char* msg, size_t n) {
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(16) << 20;   // 16 MiB
+constexpr size_t kNoallocReady = 32768;                       // up-item flags at most
+constexpr size_t kNoallocCnt = 65536;                         // counters per bank at most
+// Zero-initialised: the decode kernel's launch sequence number, flags and
+// counters at fixed offsets at the start, then the per-launch buffers.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 __device__ int g_noalloc_err_sink[4];                        // errors when err == NULL
-// Grid-barrier state of the decode kernel: it must start at zero and every
-// launch leaves it at zero again.
-__device__ unsigned int g_noalloc_gbar[4] = {0u, 0u, 0u, 0u};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 
 // Per-device set-up on the first call (that device current): the device
-// addresses of the scratch array, the error sink and the barrier state, the
-// SM count, the opt-in shared memory, and the kernels' shared-memory
-// attribute.
+// addresses of the scratch array and the error sink, the SM count, the
+// opt-in shared memory, and the kernel's shared-memory attribute.
 struct NoallocDevice {
     void* scratch;
     int* sink;
-    unsigned int* gbar;
     int sm_count;
     int smem_limit;
 };
@@ -859,17 +864,14 @@ bool noalloc_setup(int dev, NoallocDevice* out) {
     if (!d.scratch) {
         void* p = nullptr;
         void* q = nullptr;
-        void* gb = nullptr;
         int sms = 0, optin = 0;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return false;
         if (cudaGetSymbolAddress(&q, g_noalloc_err_sink) != cudaSuccess) return false;
-        if (cudaGetSymbolAddress(&gb, g_noalloc_gbar) != cudaSuccess) return false;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
         optin -= 1024;
-        if (allow_decode_smem_all(optin) != cudaSuccess) return false;
+        if (allow_mx_smem(optin) != cudaSuccess) return false;
         d.sink = static_cast<int*>(q);
-        d.gbar = static_cast<unsigned int*>(gb);
         d.sm_count = sms;
         d.smem_limit = optin;
         d.scratch = p;
@@ -878,7 +880,6 @@ bool noalloc_setup(int dev, NoallocDevice* out) {
     return true;
 }
 
-inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 }  // namespace
 
@@ -897,21 +898,21 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
         return MOE_FP4_EINVAL;
     const size_t H = cfg->hidden, I = cfg->inter, k = cfg->top_k, E = cfg->n_experts;
     const size_t ent = static_cast<size_t>(T) * k;
-    // scratch: x rows (f16) and their scales, h rows (f16) and block scales,
-    // per-entry outputs, combine counters
-    const size_t o_xh = 0, o_xs = align256(o_xh + T * H * 2), o_hh = align256(o_xs + T * 4);
-    const size_t o_hs = align256(o_hh + ent * I * 2), o_o = align256(o_hs + ent * (I / 32) * 4);
-    const size_t o_tc = align256(o_o + ent * H * 4), need = o_tc + (H / 16) * 4;
-    if (need > kNoallocScratchBytes) return MOE_FP4_EINVAL;
     const SlotLayout L = make_slot_layout(cfg->hidden, cfg->inter);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_FP4_ECUDA;
     NoallocDevice d{};
     if (!noalloc_setup(dev, &d)) return MOE_FP4_ECUDA;
-    const DecodePlan p = make_decode_plan(L, T, static_cast<int>(k), static_cast<int>(E), false, d.smem_limit, d.sm_count);
+    // scratch: the persistent header, the decode workspace of this batch, per-entry outputs
+    const MxSizes z = mx_sizes(L, T, static_cast<int>(k), static_cast<int>(E), d.sm_count);
+    const MxOffsets o = mx_offsets(z, kNoallocReady * 4, kNoallocCnt * 4);
+    const size_t o_o = o.total, need = o_o + ent * H * 4;
+    if (need > kNoallocScratchBytes || z.ready > kNoallocReady * 4 || z.cnt > kNoallocCnt * 4) return MOE_FP4_EINVAL;
+    const MxPlan p = make_mx_plan(L, T, static_cast<int>(k), static_cast<int>(E), false, d.smem_limit);
     if (!p.ok) return MOE_FP4_EINVAL;                         // shape or batch the decode kernel does not take
     uint8_t* sp = static_cast<uint8_t*>(d.scratch);
-    DecodeArgs a{};
+    MxArgs a{};
+    mx_bind(&a, sp, o, kNoallocCnt * 4);
     a.arena = arena;
     a.slot_bytes = moe_fp4_slot_bytes(cfg);
     a.slot_table = slot_table;
@@ -925,20 +926,14 @@ extern "C" moe_fp4_status moe_fp4_forward_noalloc(const moe_fp4_config* cfg, con
     a.offsets = const_cast<int32_t*>(offsets);
     a.perm = const_cast<int32_t*>(perm);
     a.x = x;
-    a.xh = reinterpret_cast<uint16_t*>(sp + o_xh);
-    a.xs = reinterpret_cast<float*>(sp + o_xs);
-    a.hh = reinterpret_cast<uint16_t*>(sp + o_hh);
-    a.hs = sp + o_hs;
     a.obuf = reinterpret_cast<float*>(sp + o_o);
-    a.tile_cnt = reinterpret_cast<int*>(sp + o_tc);
-    a.gbar = d.gbar;
-    const bool fuse = T <= kDecCombineMax;                    // else the combine kernel follows
+    const bool fuse = T <= kMxCombineMax;                     // else the combine kernel follows
     a.y = fuse ? y : nullptr;
     a.x_out = fuse ? x_out : nullptr;
     a.err = err ? reinterpret_cast<int*>(err) : d.sink;
     a.timeout_ns = 1000000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (launch_decode(a, L, p, d.sm_count, s) != cudaSuccess) return MOE_FP4_ECUDA;
+    if (launch_mx(a, L, p, d.sm_count, s) != cudaSuccess) return MOE_FP4_ECUDA;
     if (!fuse) {
         const int n4 = T * static_cast<int>(H / 4);
         if (launch_pdl(combine_kernel, dim3((n4 + 255) / 256), dim3(256), 0, s, static_cast<const float*>(a.obuf),

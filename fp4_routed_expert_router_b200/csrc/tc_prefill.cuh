@@ -17,10 +17,10 @@
 // stage (128 K, two 128-byte swizzle atoms).  One persistent CTA per SM, warp
 // roles:
 //   warps 0-15   dequantisers: warp w works in TMEM lane group w % 4 and
-//                takes lane column c = w / 4 of every 128-K stage: each
-//                thread reads its row's 16-byte chunk c (codes 8c .. 8c+7 of
-//                the four 32-K blocks, slot_layout.cuh), converts them to f16
-//                (exact E2M1), multiplies each block by 2^(s - s_ref) with
+//                takes 32-K block c = w / 4 of every 128-K stage: each
+//                thread reads its row's 16-byte chunk of block c (32 codes,
+//                slot_layout.cuh) and the block's scale byte, converts the
+//                codes to f16 (exact E2M1), multiplies them by 2^(s - s_ref) with
 //                s_ref the row's largest scale (exact while the row's scales
 //                span at most 24 binades: f16 reaches 2^-24), and writes them
 //                to the stage's A columns in TMEM with tcgen05.st (lane =
@@ -34,8 +34,10 @@
 //                gathered token rows (x grouped by expert, or h, both as f16
 //                with an exact power-of-two prescale per row), 128-byte
 //                swizzle, into shared memory.
-//   warp 21      code producer: cp.async.bulk of the item's slot blocks (all
-//                of its rows for one block's K = two stages) into a ring.
+//   warp 21      code producer: cp.async.bulk of the item's rows of one
+//                128-K unit per stage (up: rows 64h.. of the w1 and the w3
+//                unit and both scale atoms; down: the whole w2 unit) into a
+//                ring.
 //   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 (f16 x f16)
 //                with A from TMEM and B from shared memory (fp32 accumulate
 //                in TMEM), eight
@@ -140,14 +142,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 4 consecutive 32-bit columns of this thread's TMEM lane (no wait).
-__device__ __forceinline__ void tmem_st4_nowait(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
-                 "r"(r3)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // f16x2 product (exact here: a power of two times an E2M1 value).
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -213,8 +207,7 @@ __global__ void __launch_bounds__(256) h_convert_kernel(const uint16_t* hb, int 
 template <bool UP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
-    constexpr int MATS = UP ? 2 : 1;             // code matrices in a slot block
-    constexpr int ROWT = UP ? 4 : 8;             // slot row tiles (16 rows) per item
+    constexpr int ROWT = UP ? 4 : 8;             // 16-row groups per item
     constexpr int OUT_ROWS = UP ? 64 : 128;      // output rows per item
     constexpr int ACOLS = kTcSK / 2;             // TMEM columns of one stage's A (bf16 pairs)
     constexpr int BATOM = kTcNmax * 128;         // bytes of one B swizzle atom (N rows x 64 K)
@@ -247,12 +240,8 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     const int E = a.E;
     const int K = UP ? a.H : a.I;
     const int n_mt = (UP ? a.I : a.H) / OUT_ROWS;
-    const int KB = UP ? L.KBu : L.KBd;           // K of one slot block = one code entry
-    const int nfb = K / KB;                      // entries per item
-    const int spe = KB / kTcSK;                  // stages per entry
-    const int n_stg = nfb * spe;                 // stages per item
-    const size_t BB = UP ? L.UB : L.DB;          // bytes of one slot block
-    const int rbb = KB / 2, sbb = KB / 32;      // code / scale bytes of a block row
+    const int nfb = K / kTcSK;                   // code entries (= stages) per item: one 128-K unit each
+    const int n_stg = nfb;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -350,57 +339,57 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
 
     if (warp < kTcDequantWarps) {
         // ------------------------------------------------------------ dequantisers
-        // Warp w works in TMEM lane group w % 4 and lane column c = w / 4:
-        // per 128-K stage each thread converts its row's chunk c (eight codes
-        // of each of the four 32-K blocks) and stores four 4-column pieces.
-        const int cc = warp >> 2;                              // lane column of the stage
-        const int rr = lane & 15;                              // row inside the slot block
-        const int blk = UP ? lg : 2 * lg + (lane >> 4);        // slot block of the entry
-        const int mat = UP ? (lane >> 4) : 0;                  // w1 / w3 half of an up block
-        const int code_off = blk * static_cast<int>(BB) + mat * 16 * rbb + rr * rbb;
-        const int scale_off = blk * static_cast<int>(BB) + MATS * 16 * rbb + mat * 16 * sbb + rr * sbb;
-        int gstg = 0, gentry = 0;
+        // Warp w works in TMEM lane group w % 4 and takes 32-K block c = w / 4
+        // of every 128-K stage: each thread converts its row's 32 codes of
+        // block c (one 16-byte chunk of the unit, slot_layout.cuh), scales
+        // them by 2^(s - s_ref) and stores 16 columns (K in natural order).
+        const int cc = warp >> 2;                              // 32-K block of the stage
+        // up: lanes 0-15 w1 rows, 16-31 w3 rows of the item's 64; down: row 32 lg + lane
+        const int mat = UP ? (lane >> 4) : 0;
+        const int rloc = UP ? 16 * lg + (lane & 15) : 32 * lg + lane;
+        int gstg = 0;
         for (int i = 0; i < my_items; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int slot = act_slot[ai];
             if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[ai], kid);
+            // entry layout: up  [w1 rows 64h.. codes 4096][w3 codes 4096][w1 scale atom][w3 scale atom]
+            //               down [the unit, 8704]
+            const int urow = UP ? 64 * (mt & 1) + rloc : rloc;       // row inside the 128-row unit
+            const int code_off = UP ? mat * 4096 + unit_code_chunk(rloc, cc) : unit_code_chunk(rloc, cc);
+            const int scale_off = UP ? 2 * 4096 + mat * kUnitScaleBytes + unit_scale_byte(urow, cc) - kUnitCodeBytes
+                                     : unit_scale_byte(urow, cc);
             // the row's largest scale (load-time table)
-            const int wrow = UP ? (mt * ROWT + lg) * 16 + rr : (mt * ROWT + blk) * 16 + rr;
+            const int wrow = mt * OUT_ROWS + rloc;
             const int sref = slot < 0 ? 0
                                       : __ldg(t.rowref + static_cast<size_t>(slot) * (2 * a.I + a.H) +
                                               (UP ? mat * a.I : 2 * a.I) + wrow);
-            for (int f = 0; f < nfb; ++f, ++gentry) {
-                const int ce = gentry % CE;
-                if (!mbar_wait(&cfull[ce], (gentry / CE) & 1, abort_flag, t.timeout_ns) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gentry, kid);
+            for (int f = 0; f < nfb; ++f, ++gstg) {
+                const int ce = gstg % CE;
+                if (!mbar_wait(&cfull[ce], (gstg / CE) & 1, abort_flag, t.timeout_ns) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
                 const uint8_t* ent = code_entry(ce);
-                for (int j = 0; j < spe; ++j, ++gstg) {
-                    const int st = gstg % S;
-                    if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
-                        latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
-                    tc_fence_after();
-                    // stage j = 128-K group j of the block row
-                    const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off +
-                                                                    swizzle_chunk(4 * j + cc, rr, rbb) * 16);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t*>(ent + scale_off + 4 * j);
-                    const uint32_t col0 = tmem_a + lane_addr + st * ACOLS + 4 * cc;
+                const int st = gstg % S;
+                if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                tc_fence_after();
+                const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off);
+                const int sq = ent[scale_off];
+                const uint32_t mult = (slot < 0) ? 0u : mtab[(sref - sq) & 255];
+                uint32_t o[16];
+                e2m1x8_to_f16x2(w.x, o);
+                e2m1x8_to_f16x2(w.y, o + 4);
+                e2m1x8_to_f16x2(w.z, o + 8);
+                e2m1x8_to_f16x2(w.w, o + 12);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {   // 32-K block q of the group: K = 32q + 8cc .. +7
-                        const int sq = static_cast<int>(__byte_perm(sw, 0u, 0x4440u | static_cast<uint32_t>(q)));
-                        const uint32_t mult = (slot < 0) ? 0u : mtab[(sref - sq) & 255];
-                        uint32_t o[4];
-                        e2m1x8_to_f16x2(q == 0 ? w.x : q == 1 ? w.y : q == 2 ? w.z : w.w, o);
-                        tmem_st4_nowait(col0 + 16 * q, hmul2_u32(o[0], mult), hmul2_u32(o[1], mult),
-                                        hmul2_u32(o[2], mult), hmul2_u32(o[3], mult));
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full[st]);
-                }
+                for (int q = 0; q < 16; ++q) o[q] = hmul2_u32(o[q], mult);
+                tmem_st16(tmem_a + lane_addr + st * ACOLS + 16 * cc, o);
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cfree[ce]);
+                if (lane == 0) {
+                    mbar_arrive(&full[st]);
+                    mbar_arrive(&cfree[ce]);
+                }
             }
         }
     } else if (warp < kTcDequantWarps + kTcEpiWarps) {
@@ -520,13 +509,20 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                 if (lane == 0) {
                     if (slot < 0) {
                         mbar_arrive(&cfull[ce]);
+                    } else if (UP) {   // rows 64h .. 64h+63 of the w1 and w3 units (rt, f), and both scale atoms
+                        const int rt = mt >> 1, hh = mt & 1;
+                        const uint8_t* u1 = src + up_unit_offset(L, 0, rt, f);
+                        const uint8_t* u3 = src + up_unit_offset(L, 1, rt, f);
+                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(t.entry_bytes));
+                        bulk_g2s(code_entry(ce), u1 + 4096 * hh, 4096u, &cfull[ce], pol);
+                        bulk_g2s(code_entry(ce) + 4096, u3 + 4096 * hh, 4096u, &cfull[ce], pol);
+                        bulk_g2s(code_entry(ce) + 8192, u1 + kUnitCodeBytes, kUnitScaleBytes, &cfull[ce], pol);
+                        bulk_g2s(code_entry(ce) + 8192 + kUnitScaleBytes, u3 + kUnitCodeBytes, kUnitScaleBytes,
+                                 &cfull[ce], pol);
                     } else {
-                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(ROWT * BB));
-                        for (int b = 0; b < ROWT; ++b) {   // the item's row tiles, block f
-                            const size_t rt = static_cast<size_t>(mt) * ROWT + b;
-                            bulk_g2s(code_entry(ce) + b * BB, src + (rt * nfb + f) * BB,
-                                     static_cast<uint32_t>(BB), &cfull[ce], pol);
-                        }
+                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(kUnitBytes));
+                        bulk_g2s(code_entry(ce), src + down_unit_offset(L, mt, f) - L.up_bytes, kUnitBytes,
+                                 &cfull[ce], pol);
                     }
                 }
                 __syncwarp();
@@ -678,12 +674,11 @@ inline TcArgs tc_args(const TcPlan& p, const ExpertArgs& g, const SlotLayout& L,
     const int head = 1024 + 256 * 16 + 4 * (5 * t.max_active + 1 + 2 * g.E + 1);
     t.off_b = (head + 1023) / 1024 * 1024;
     t.off_code = t.off_b + kTcStages * 2 * kTcNmax * 128;
-    t.entry_bytes = static_cast<int>(up ? 4 * L.UB : 8 * L.DB);
+    t.entry_bytes = up ? 2 * (4096 + kUnitScaleBytes) : kUnitBytes;
     int ce = (p.smem_limit - 1024 - t.off_code) / t.entry_bytes;
     if (ce > kTcMaxEntries) ce = kTcMaxEntries;
     const int K = up ? g.H : g.I, rows = up ? g.I : g.H;
-    const int KBk = up ? L.KBu : L.KBd;
-    const bool shape_ok = (K % kTcSK == 0) && (KBk % kTcSK == 0) && (rows % (up ? 64 : kTcM) == 0);
+    const bool shape_ok = (K % kTcSK == 0) && (rows % kTcM == 0);
     t.centries = (ce >= 2 && shape_ok) ? ce : 0;
     return t;
 }

@@ -49,6 +49,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// Same without an L2 eviction hint (small operands that other CTAs read too).
+__device__ __forceinline__ void bulk_g2s_nohint(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // One bounded probe of phase `parity`: the hardware may suspend the thread
 // for up to `hint_ns` (at most ~0.5 ms) waiting for the phase instead of a
 // hot spin.
@@ -81,6 +88,32 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// Raise the transaction count of the current phase by `bytes` without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Wait for phase `parity` of `bar` by polling (non-blocking probes with a
+// short sleep between them): the phase is seen within tens of nanoseconds
+// whichever agent completes it.  Same bounds and abort rules as mbar_wait.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t timeout_ns = 1000000000ull) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+        __nanosleep(32);
+        if (mbar_test(bar, parity)) return true;
+        if ((n & 15) == 0) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > timeout_ns) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
 }
 
 // Wait for phase `parity` of `bar` to complete.  Returns false at once when

@@ -323,31 +323,37 @@ moe_fp4_status moe_fp4_last_error(moe_fp4_ctx *ctx, char *msg, size_t n);
 
 /*
  * Forward without any allocation: the same decode kernel as moe_fp4_forward
- * (the whole layer in one launch: grouped GEMV, SwiGLU, combine), for callers
- * that cannot call cudaMalloc -- for example a plugin inside a host framework
- * that owns all device memory and forbids allocation on its execution path,
- * or code that runs where the CUDA allocator must not be entered.  This call
- * has no counterpart on the pages: it is a deployment variant of this library.
+ * (the whole layer in one launch: both expert GEMMs on the block-scaled FP4
+ * tensor cores, SwiGLU, combine), for callers that cannot call cudaMalloc --
+ * for example a plugin inside a host framework that owns all device memory
+ * and forbids allocation on its execution path, or code that runs where the
+ * CUDA allocator must not be entered.  This call has no counterpart on the
+ * pages: it is a deployment variant of this library.
  *
  * Nothing is allocated and no context is used.  The caller passes every input
- * and output; the forward's scratch (prescaled f16 x and h rows with their
- * scales, fp32 per-entry outputs, the combine counters) lives in one
- * library-owned, file-scope device array of 16 MiB (16,777,216 bytes) that
- * every GPU which loads the library holds until the process exits, next to
- * 16 bytes of grid-barrier state.  The scratch must hold
- *   T*H*2 + T*4 + T*k*I*2 + T*k*(I/32)*4 + T*k*H*4 + (H/16)*4 bytes
- * (each part rounded up to 256); a larger T, or a shape the decode kernel
- * does not take, returns EINVAL before any launch.  For the V4.1 shape (k = 6)
- * that allows T <= 103.  Up to 16 tokens the combine runs inside the kernel,
- * above that a second kernel.
+ * and output; the forward's scratch lives in one library-owned, file-scope
+ * device array of 16 MiB (16,777,216 bytes) that every GPU which loads the
+ * library holds until the process exits.  It starts with a fixed header of
+ * 656,640 bytes (the kernel's launch sequence number, 1 KB of zeros, up to
+ * 32,768 up-item flags and two banks of 65,536 counters, all zero at load and
+ * kept consistent by every launch), followed by the per-call buffers: the digit
+ * planes of x and h with their scales, split-item partial sums and fp32
+ * per-entry outputs.  With KU = H/128, KD = I/128 and S the device's SM count
+ * the scratch must hold
+ *   656640 + T*KU*512 + T*KU*128 + T*k*KD*512 + T*k*KD*128 + S*6144 + T*k*H*4
+ * bytes (each of the five middle parts rounded up to 256), and the batch's
+ * work items must fit the header (max_gs*(I/128) flags and
+ * 1 + max_gs*(I/128 + H/128) + H/128 counters per bank, max_gs = min(T*k, min(E, T*k)
+ * + T*k/2)); a larger T, or a shape the decode kernel does not take, returns
+ * EINVAL before any launch.  For the V4.1 shape (k = 6) on a 148-SM B200 that
+ * allows T <= 69.  Up to 16 tokens the combine runs inside the kernel, above
+ * that a second kernel.
  *
  * Every call, on every stream, shares that array and leaves the last call's
- * contents in it; the kernel itself clears what must start at zero (the
- * combine counters) and leaves the barrier state at zero.  Calls whose
- * executions overlap on the GPU race on it: serialise them (one stream, or
- * events).  The first call on a device looks up the array's device address
- * with cudaGetSymbolAddress (once per device, that device current); make that
- * first call before any stream capture.
+ * contents in it.  Calls whose executions overlap on the GPU race on it:
+ * serialise them (one stream, or events).  The first call on a device looks
+ * up the array's device address with cudaGetSymbolAddress (once per device,
+ * that device current); make that first call before any stream capture.
  *
  *  cfg         the layer shape (as for moe_fp4_create; n_slots and max_tokens
  *              only bound the indices used).
