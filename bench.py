@@ -13,7 +13,9 @@ experts resident and the rest streamed from pinned host memory, then the
 40-layer stack (batch 1 and 8, its own 115.8 GB arena), all reported under
 "workloads".
 Inputs are resident in HBM when a timed step starts; L2 is flushed between
-timed steps (a 2x L2-sized write), so expert bytes really come from HBM.
+timed steps (a 2x L2-sized write whose lines are then discarded), so expert
+bytes really come from HBM, and the step's small inputs (x, logits) are
+written after the flush, as the preceding layer of a model leaves them.
 Rank 0 prints one JSON line.  Under torchrun each rank runs an independent
 replica (data parallel, no collective on the data path): weak scaling.
 
@@ -62,7 +64,9 @@ def workload_config(wl: synth.Workload, graph: bool) -> dict:
         "expert_bytes": wl.expert_bytes, "weights": "fp4 e2m1 + ue8m0 per 32 along K",
         "logits": f"N(0,1) + Zipf(1.1) bias, alpha {wl.zipf_alpha}",
         "scale_exponents": f"uniform {wl.scale_lo}..{wl.scale_hi}",
-        "l2": "flushed between timed steps (2x L2 write, then its lines discarded)",
+        "l2": "flushed between timed steps (2x L2 write, then its lines discarded); the step's small inputs "
+              "(x, logits) are written after the flush, as the preceding layer leaves them, the expert "
+              "weights come from HBM",
         "launch": ("cuda graph of moe_fp4_route_forward" if graph else "eager moe_fp4_route_forward") +
                   (" (one persistent kernel per step)" if wl.tokens * wl.top_k <= 64 else
                    " (route kernel, then the expert kernels)"),
@@ -282,10 +286,10 @@ class Bench:
         def step_launch():
             ctx.route_forward(0, l_buf, x_buf, out=routing, y=y_buf, stream=stream)
 
-        def stage(i):
+        def stage(i):   # L2 flushed, then the step's inputs written (as the preceding layer leaves them)
+            moe.l2_flush(flush, float(i), stream)
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
             l_buf.copy_(pool_l[i % npool], non_blocking=True)
-            moe.l2_flush(flush, float(i), stream)
 
         out = {}
         graph = None
@@ -424,10 +428,10 @@ def run_stack(wls, local, rank, steps, warmup, graph_ok, peaks, world, dist):
                 ctx.route_forward(l, l_buf[l], x_buf, keep=masks[l], out=routes[l], y=y_buf, x_out=x_buf,
                                   stream=stream)
 
-        def stage(i):
+        def stage(i):   # L2 flushed, then the step's inputs written (as the preceding layer leaves them)
+            moe.l2_flush(flush, float(i), stream)
             x_buf.copy_(pool_x[i % npool], non_blocking=True)
             l_buf.copy_(pool_l[i % npool], non_blocking=True)
-            moe.l2_flush(flush, float(i), stream)
 
         graph = None
         with torch.cuda.stream(stream):

@@ -35,10 +35,9 @@
 // another; an item cut by a range boundary is finished by whichever of its
 // CTAs completes last, which adds the fp32 partials in CTA order (results do
 // not depend on timing).  Inside a CTA:
-//   warps 7-15, lane 0  producers: bulk copies of unit i (A + scales from the
-//                       arena, B + B scales from the plane buffers) into ring
-//                       slot i % S, warp 7 + i % 9 per unit (S a multiple of
-//                       9, so a slot always has the same producer and issuer);
+//   warps 10-15         producers, one lane per ring slot (S / 6 lanes each):
+//                       bulk copies of unit i (A + scales from the arena, B +
+//                       B scales from the plane buffers) into slot i % S;
 //   warps 4-6, lane 0   MMA issuers: issuer i % 3 takes unit i -- tcgen05.cp
 //                       of both scale atoms into its own TMEM columns, two
 //                       K = 64 MMAs into its own double-buffered accumulator,
@@ -76,26 +75,31 @@ constexpr int kMxThreads = kMxWarps * 32;
 constexpr int kMxEpiWarps = 4;                    // warps 0-3: TMEM lane quadrant = warp
 constexpr int kMxMmaWarp = 4;                     // warps 4 .. 9: one MMA issuer lane each
 constexpr int kMxIssuers = 6;
-constexpr int kMxProdWarp = kMxMmaWarp + kMxIssuers;   // warps 10 .. 15: one producer lane each
-constexpr int kMxProducers = kMxWarps - kMxProdWarp;
-// Ring slots come in multiples of this: slot s is then always filled by
-// producer s % 6 and drained by issuer s % 6, so each thread sees the uses of
+constexpr int kMxProdWarp = kMxMmaWarp + kMxIssuers;   // warps 10 .. 15: S / 6 producer lanes each
+constexpr int kMxProdWarps = kMxWarps - kMxProdWarp;
+// Ring slots come in multiples of this: slot s is always filled by its own
+// producer lane and drained by issuer s % 6, so each thread sees the uses of
 // its slots in order and every mbarrier parity wait is unambiguous.
-constexpr int kMxSlotQuantum = 6;
-static_assert(kMxSlotQuantum % kMxProducers == 0 && kMxSlotQuantum % kMxIssuers == 0, "slot ownership");
+constexpr int kMxSlotQuantum = kMxIssuers;
+static_assert(kMxProdWarps == kMxIssuers, "one producer lane per slot: S / 6 lanes in each of 6 warps");
 constexpr int kMxGroup = 2;                       // entries per token group: N = 8 * entries <= 16
 constexpr int kMxPlanes = 8;                      // E2M1 digit planes per activation row
 constexpr int kMxPlaneTile = 512;                 // one row's planes for 128 K: [4 blocks][8 planes][16 B]
 constexpr int kMxPlaneScale = 128;                // their scales: [8 planes][16 B], byte b = block b
 constexpr int kMxOffB = kUnitBytes;               // slot: A codes | A scales | B (g x 512) | B scale rows (g x 128)
 constexpr int kMxMaxSlots = 24;
+constexpr int kMxPrefetchLaps = 0;                // weights prefetched into L2 this many ring laps ahead
+                                                  // (0: none -- two laps measured slower at batch 1 on B200)
 constexpr int kMxRouteMax = 64;                   // T*k routed inside the kernel at most
 constexpr int kMxRouteExperts = 384;              // E routed inside the kernel at most
 constexpr int kMxCombineMax = 16;                 // tokens combined inside the kernel at most
 constexpr int kMxMaxEntries = 768;                // token-expert entries of one launch at most (workspace)
-constexpr int kMxPartFloats = 3 * 2 * kMxGroup * 128;   // per CTA: up 2 sides x 2 mats, down 2 sides
-constexpr int kMxPartUp = 2 * kMxGroup * 128;            // floats of one up side (w1 then w3)
-constexpr int kMxPartDown = kMxGroup * 128;              // floats of one down side
+constexpr int kMxChunks = 1;                      // chunks of token groups in the schedule (see the work section)
+constexpr int kMxLag = 2;                         // down(c) runs after up(c + kMxLag)
+constexpr int kMxPartUp = 2 * kMxGroup * 128;     // floats of one up side (w1 then w3)
+constexpr int kMxPartDown = kMxGroup * 128;       // floats of one down side
+constexpr int kMxPartChunk = 2 * kMxPartUp + 2 * kMxPartDown;   // per chunk: 2 up sides, 2 down sides
+constexpr int kMxPartFloats = kMxChunks * kMxPartChunk;         // split-item partials of one CTA
 constexpr uint32_t kMxTmemCols = 512;             // accumulators [2][issuer][16 g] columns, scale atoms at 384 + 8 w
 
 struct MxArgs {
@@ -190,6 +194,46 @@ __device__ __forceinline__ float mx_ld8_sum(uint32_t taddr) {
     return s;
 }
 
+// 8 or 16 consecutive fp32 TMEM columns of this thread's lane into r[0 .. n), no wait.
+__device__ __forceinline__ void mx_ld_issue16(uint32_t taddr, int n, uint32_t (&r)[16]) {
+    if (n == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+    }
+}
+
+// n (8, 16 or 32) consecutive fp32 TMEM columns of this thread's lane into r[0 .. n).
+__device__ __forceinline__ void mx_ld_cols(uint32_t taddr, int n, uint32_t (&r)[32]) {
+    if (n == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+    } else if (n == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+              "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+              "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+            : "r"(taddr));
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void mx_named_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -211,6 +255,13 @@ __device__ __forceinline__ void mx_st_release(unsigned int* p, unsigned int v) {
 // Generic-proxy writes (by any thread, ordered before this point) become
 // visible to the async proxy (bulk copies) issued after it.
 __device__ __forceinline__ void mx_fence_proxy_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// x * 2^e, exact whenever the result is representable (two multiplies by
+// normal powers of two; -252 <= e <= 254).
+__device__ __forceinline__ float mx_mul_pow2(float x, int e) {
+    const int e1 = e / 2, e2 = e - e1;
+    return (x * __uint_as_float(static_cast<uint32_t>(e1 + 127) << 23)) * __uint_as_float(static_cast<uint32_t>(e2 + 127) << 23);
+}
 
 // Split one 32-element block (v = this lane's element, a bf16 value held in
 // fp32) into kMxPlanes E2M1 digit planes: plane p -> 16 bytes at pc + 16 p
@@ -238,10 +289,10 @@ __device__ __forceinline__ void mx_split_block(float v, int lane, uint8_t* pc, u
         uint32_t code = 0u;
         int sbyte = 0;
         if (live && s >= -127) {
-            const float d = rintf(2.0f * ldexpf(r, -s)) * 0.5f;   // nearest half: |d| <= 2
+            const float d = rintf(2.0f * mx_mul_pow2(r, -s)) * 0.5f;   // nearest half: |d| <= 2
             const float ad = fabsf(d);
             code = static_cast<uint32_t>(2.0f * ad) | (d < 0.0f ? 8u : 0u);
-            r -= ldexpf(d, s);                  // exact: |r| shrinks below 2^(s-2)
+            r -= mx_mul_pow2(d, s);             // exact: |r| shrinks below 2^(s-2)
             sbyte = s + 127;
         } else if (!live && p == 0 && mb != 0u) {
             sbyte = 255;
@@ -306,35 +357,33 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
     const int n_ent = a.T * k;
     const int KU = L.KU, KD = L.KD, RT = L.RT, NT = L.NT;
 
-    if (tid == 0) {
-        tag_s = mx_ld_acquire(a.seq) + 1u;   // this launch's tag (never 0 for 2^32 launches)
-        for (int s = 0; s < kMxMaxSlots; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int q = 0; q < 2; ++q) {
-            mbar_init(&accf[q], kMxIssuers);
-            mbar_init(&acce[q], kMxEpiWarps);
-        }
-        for (int q = 0; q < kMxIssuers; ++q) mbar_init(&fin[q], 1);
-        for (int s = 0; s < kMxMaxSlots; ++s) last_issue[s] = -1;
-        abort_s = 0;
-        fence_barrier_init();
-    }
+    // Set-up runs beside the first loads: lane 0 of the TMEM warp reads the
+    // launch sequence number and initialises the barriers, the warp allocates
+    // TMEM, a producer warp reads the slot table row, and from the first
+    // instruction the other warps route (below) and make x planes.
     if (warp == kMxMmaWarp) {
+        if (lane == 0) {
+            tag_s = mx_ld_acquire(a.seq) + 1u;   // this launch's tag (never 0 for 2^32 launches)
+            for (int s = 0; s < kMxMaxSlots; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int q = 0; q < 2; ++q) {
+                mbar_init(&accf[q], kMxIssuers);
+                mbar_init(&acce[q], kMxEpiWarps);
+            }
+            for (int q = 0; q < kMxIssuers; ++q) mbar_init(&fin[q], 1);
+            for (int s = 0; s < kMxMaxSlots; ++s) last_issue[s] = -1;
+            abort_s = 0;
+            fence_barrier_init();
+        }
+        __syncwarp();
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_s)),
                      "r"(kMxTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (warp == kMxProdWarp)   // this layer's slot table row
         for (int e = lane; e < E; e += 32) slot_s[e] = __ldg(a.slot_table + static_cast<size_t>(a.layer) * E + e);
-
-    // the counter bank of the next launch starts at zero
-    {
-        const unsigned int nb = (mx_ld_acquire(a.seq) + 2u) & 1u;   // bank of launch seq + 1
-        unsigned int* other = a.cnt + static_cast<size_t>(nb) * a.cnt_cap;
-        for (int i = b * kMxThreads + tid; i < a.cnt_cap; i += G * kMxThreads) other[i] = 0u;
-    }
 
     // ------------------------------------------------------------ x digit planes (a share per warp)
     {
@@ -349,11 +398,25 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
     }
 
     // ------------------------------------------------------------ routing
+    // x planes, routing and set-up done: count this CTA's planes on the launch's
+    // x counter (the copies of x planes wait for every CTA), clear the counter
+    // bank of the next launch
+    auto after_first_sync = [&]() {
+        if (tid == kMxThreads - 32) {   // not warp 0, which groups the entries next
+            __threadfence();
+            mx_fence_proxy_global();
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;"
+                         ::"l"(a.cnt + static_cast<size_t>(tag_s & 1u) * a.cnt_cap) : "memory");
+        }
+        unsigned int* other = a.cnt + static_cast<size_t>((tag_s + 1u) & 1u) * a.cnt_cap;
+        for (int i = b * kMxThreads + tid; i < a.cnt_cap; i += G * kMxThreads) other[i] = 0u;
+    };
     if (routed) {
         for (int t = warp; t < a.T; t += kMxWarps)
             route_one<kMxRouteExperts / 32>(a.logits + static_cast<size_t>(t) * E, a.keep, E, k, t, lane,
                                            r_ids + t * k, r_w + t * k, a.err);
         __syncthreads();
+        after_first_sync();
         if (warp == 0) {
             // stable grouping of the <= 64 entries by expert: rank of key (expert, entry)
 #pragma unroll
@@ -408,6 +471,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
     } else {
         for (int e = tid; e <= E; e += blockDim.x) offs_s[e] = __ldg(a.offsets + e);
         __syncthreads();
+        after_first_sync();
         if (warp == 0) {
             int n = 0;
             for (int base = 0; base < E; base += 32) {
@@ -430,12 +494,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
             if (lane == 0) n_act_s = min(n, p.max_act);
         }
         __syncthreads();
-    }
-    // x planes of this CTA stored: count it (the copies of x planes wait for every CTA)
-    if (tid == 0) {
-        __threadfence();
-        mx_fence_proxy_global();
-        atomicAdd(a.cnt + static_cast<size_t>(tag_s & 1u) * a.cnt_cap, 1u);
     }
     const int n_act = n_act_s;
     for (int q = tid; q < n_act; q += blockDim.x) act_slot[q] = slot_s[act_e[q]];
@@ -467,16 +525,18 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
     mx_fence_after();
 
     // ------------------------------------------------------------ work
+    // The groups form C = min(n_gs, kMxChunks) chunks; each chunk's up units,
+    // and its down units, are split contiguously over all CTAs, and every CTA
+    // runs its segments in the order up(0) .. up(L-1), then up(c), down(c - L)
+    // for c = L .. C-1, then the last L downs.  With kMxChunks = 1 (the setting
+    // used) that is all up units, then all down units: a staggered order with
+    // six chunks measured 3.4x slower at batch 1 on B200, because accumulators
+    // and the epilogue run strictly in order, so a down part waiting for
+    // another CTA's h holds up every part queued behind it.
     const int n_gs = n_gs_s;
     const unsigned int tag = tag_s;
     const int upi = 2 * KU, dpi = KD;                       // units per up / down item
-    const int NU = n_gs * RT * upi, ND = n_gs * NT * dpi;   // units of all items
-    const int u0 = mx_range_start(NU, G, b), u1 = mx_range_start(NU, G, b + 1);
-    const int d0 = mx_range_start(ND, G, b), d1 = mx_range_start(ND, G, b + 1);
-    const int nu = u1 - u0, n_units = nu + (d1 - d0);
-    const int up_first = nu > 0 ? u0 / upi : 0, n_up_parts = nu > 0 ? (u1 - 1) / upi - up_first + 1 : 0;
-    const int dn_first = d1 > d0 ? d0 / dpi : 0, n_dn_parts = d1 > d0 ? (d1 - 1) / dpi - dn_first + 1 : 0;
-    const int n_parts = n_up_parts + n_dn_parts;
+    const int C = min(n_gs, kMxChunks), n_seg = 2 * C;
     unsigned int* x_cnt = a.cnt + static_cast<size_t>(tag & 1u) * a.cnt_cap;   // this launch's bank
     unsigned int* up_cnt = x_cnt + 1;
     unsigned int* dn_cnt = up_cnt + p.max_up_items;
@@ -486,106 +546,185 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
         const int ent = routed ? r_perm[pos] : __ldg(a.perm + pos);
         return (ent >= 0 && ent < n_ent) ? ent : -1;
     };
-    // part j of this CTA: its item and its unit range (global unit indices)
-    auto part_of = [&](int j, bool& up, int& item, int& ua, int& ub) {
-        up = j < n_up_parts;
-        if (up) {
-            item = up_first + j;
-            ua = max(item * upi, u0);
-            ub = min((item + 1) * upi, u1);
+    // segment s: up or down, its chunk, the chunk's unit space [base, base + n)
+    // and this CTA's range [ua, ub) in it (global unit indices)
+    auto segment = [&](int sg, bool& up, int& c, int& base, int& n, int& ua, int& ub) {
+        if (C <= kMxLag) {
+            up = sg < C;
+            c = up ? sg : sg - C;
+        } else if (sg < kMxLag) {
+            up = true;
+            c = sg;
         } else {
-            item = dn_first + (j - n_up_parts);
-            ua = max(item * dpi, d0);
-            ub = min((item + 1) * dpi, d1);
+            const int t = sg - kMxLag;
+            if (t < 2 * (C - kMxLag)) {
+                up = (t & 1) == 0;
+                c = up ? kMxLag + (t >> 1) : (t >> 1);
+            } else {
+                up = false;
+                c = C - kMxLag + (t - 2 * (C - kMxLag));
+            }
+        }
+        const int g0 = n_gs * c / C, g1 = n_gs * (c + 1) / C;
+        const int per_group = up ? RT * upi : NT * dpi;
+        base = g0 * per_group;
+        n = (g1 - g0) * per_group;
+        if (up) {   // up units split evenly: an item may be cut between CTAs
+            ua = base + mx_range_start(n, G, b);
+            ub = base + mx_range_start(n, G, b + 1);
+        } else {    // whole down items: no partial sums; their weights stream while h is made
+            const int items = n / dpi;
+            ua = base + mx_range_start(items, G, b) * dpi;
+            ub = base + mx_range_start(items, G, b + 1) * dpi;
         }
     };
     const uint32_t ring_base = smem_u32(ring);
 
     if (warp >= kMxProdWarp) {
         // ------------------------------------------------------------ producers
-        // Lane 0 of producer warp w copies units w, w + 11, ...: unit i to slot
-        // i % S once the slot's previous unit has been consumed.  x planes are
-        // copied once every CTA has stored its share; h planes once their up
-        // item is done.
-        if (lane == 0) {
-            const int pw = warp - kMxProdWarp;
+        // Producer p (lane p % (S/6) of warp 10 + p / (S/6)) owns ring slot p and
+        // the CTA's units p, p + S, ... (unit i goes to slot i % S).  It never
+        // blocks on one unit (lanes of a warp run independent producers): the weights of its units are copied as far ahead
+        // as its slots allow (they depend on the routing only), and the B
+        // operand of its oldest unit without one as soon as it is ready -- the
+        // x planes once every CTA has stored its share, the h planes once their
+        // up item is done -- so during the hand-off from the up to the down
+        // GEMM the ring fills with down weights.  expect_tx without an arrive
+        // keeps a unit's phase open until its B copies are issued too.
+        const int lanes = S / kMxProdWarps;   // producer lanes per warp: one producer per slot
+        if (lane < lanes) {
+            const int pw = (warp - kMxProdWarp) * lanes + lane;   // this producer's slot
+            const int kMxProducers = S;
             const uint64_t pol = policy_evict_first();
+            // the CTA's units as segments: local index i -> global unit gu
+            int seg_first[2 * kMxChunks + 1], seg_ua[2 * kMxChunks];
+            bool seg_up[2 * kMxChunks];
+            int n_units = 0;
+            for (int sg = 0; sg < n_seg; ++sg) {
+                int c, base, n, ua, ub;
+                bool up;
+                segment(sg, up, c, base, n, ua, ub);
+                seg_first[sg] = n_units;
+                seg_ua[sg] = ua;
+                seg_up[sg] = up;
+                n_units += ub - ua;
+            }
+            seg_first[n_seg] = n_units;
+            auto unit = [&](int i, bool& up, int& gs, int& tile, int& mat, int& ku) {
+                int sg = 0;
+                while (i >= seg_first[sg + 1]) ++sg;
+                up = seg_up[sg];
+                const int gu = seg_ua[sg] + (i - seg_first[sg]);
+                const int item = up ? gu / upi : gu / dpi, v = up ? gu - item * upi : gu - item * dpi;
+                gs = up ? item / RT : item / NT;
+                tile = up ? item - gs * RT : item - gs * NT;
+                mat = up ? v / KU : 0;
+                ku = up ? v - mat * KU : v;
+            };
+            const int nm = n_units > pw ? (n_units - pw + kMxProducers - 1) / kMxProducers : 0;   // my units
+            const int ahead = S / kMxProducers;                                                // my slots
+            int mA = 0, mB = 0;            // my next unit for the weights / for the B operand
             bool x_ok = false;
             int ready_item = -1;
-            int i = pw;
-            for (; i < n_units; i += kMxProducers) {
-                const int s = i % S;
-                if (i >= S && !mbar_poll(&empty[s], ((i / S) - 1) & 1, abort_flag, a.timeout_ns)) {
-                    latch_error(a.err, ERR_ETIMEOUT, i, KID_UP);
-                    *abort_flag = 1;
-                    break;
-                }
-                const bool up = i < nu;
-                const int gu = up ? u0 + i : d0 + (i - nu);
-                const int item = up ? gu / upi : gu / dpi, v = up ? gu - item * upi : gu - item * dpi;
-                const int gs = up ? item / RT : item / NT, tile = up ? item - gs * RT : item - gs * NT;
-                const int mat = up ? v / KU : 0, ku = up ? v - mat * KU : v;
-                const int slot = act_slot[gs_a[gs]];
-                const int ng = gs_n[gs], p0 = gs_p0[gs];
-                if (slot < 0) {   // expert not resident: nothing to copy (the epilogue writes zeros)
-                    mbar_arrive(&full[s]);
-                    continue;
-                }
-                // the weights first (they depend on the routing only), then the B
-                // operand once its producers are done: expect_tx without an arrive
-                // keeps the phase open until the B copies are issued too
-                uint8_t* dst = ring + static_cast<size_t>(s) * SB;
-                const size_t uoff = up ? up_unit_offset(L, mat, tile, ku) : down_unit_offset(L, tile, ku);
-                mbar_expect_tx(&full[s], static_cast<uint32_t>(kUnitBytes));
-                bulk_g2s(dst, a.arena + static_cast<size_t>(slot) * a.slot_bytes + uoff, kUnitBytes, &full[s], pol);
-                reinterpret_cast<volatile int*>(last_issue)[s] = i;
-                bool ok = true;
-                const uint64_t t0 = global_timer_ns();
-                if (up && !x_ok) {
-                    while (mx_ld_acquire(x_cnt) < static_cast<unsigned int>(G)) {
-                        if (*abort_flag || global_timer_ns() - t0 > a.timeout_ns) { ok = false; break; }
-                        __nanosleep(64);
+            uint64_t t_idle = global_timer_ns();
+            while (mB < nm) {
+                bool progress = false;
+                while (mA < nm && mA < mB + ahead) {   // weights, as far ahead as my slots allow
+                    const int i = pw + mA * kMxProducers, s = i % S;
+                    if (i >= S && !mbar_test(&empty[s], ((i / S) - 1) & 1)) break;
+                    bool up;
+                    int gs, tile, mat, ku;
+                    unit(i, up, gs, tile, mat, ku);
+                    const int slot = act_slot[gs_a[gs]];
+                    if (slot >= 0) {   // (an expert that is not resident gets no copies; the epilogue writes zeros)
+                        const size_t uoff = up ? up_unit_offset(L, mat, tile, ku) : down_unit_offset(L, tile, ku);
+                        mbar_expect_tx(&full[s], static_cast<uint32_t>(kUnitBytes));
+                        bulk_g2s(ring + static_cast<size_t>(s) * SB, a.arena + static_cast<size_t>(slot) * a.slot_bytes + uoff,
+                                 kUnitBytes, &full[s], pol);
+                        reinterpret_cast<volatile int*>(last_issue)[s] = i;
                     }
-                    x_ok = ok;
-                } else if (!up && ready_item != gs * RT + ku) {
-                    while (mx_ld_acquire(a.ready + gs * RT + ku) != tag) {
-                        if (*abort_flag || global_timer_ns() - t0 > a.timeout_ns) { ok = false; break; }
-                        __nanosleep(64);
+                    // optional L2 prefetch of this slot's unit kMxPrefetchLaps laps ahead (and, on the
+                    // first lap, of every lap up to that)
+                    for (int d = (mA == 0 ? 1 : kMxPrefetchLaps); kMxPrefetchLaps > 0 && d <= kMxPrefetchLaps; ++d) {
+                        const int jd = i + d * S;
+                        if (jd >= n_units) break;
+                        bool upd;
+                        int gsd, tiled, matd, kud;
+                        unit(jd, upd, gsd, tiled, matd, kud);
+                        const int sld = act_slot[gs_a[gsd]];
+                        if (sld >= 0)
+                            bulk_prefetch_l2(a.arena + static_cast<size_t>(sld) * a.slot_bytes +
+                                                 (upd ? up_unit_offset(L, matd, tiled, kud) : down_unit_offset(L, tiled, kud)),
+                                             kUnitBytes);
                     }
-                    if (ok) ready_item = gs * RT + ku;
+                    ++mA;
+                    progress = true;
                 }
-                if (!ok) {
-                    latch_error(a.err, ERR_ETIMEOUT, 200 + (up ? 0 : 1), up ? KID_UP : KID_DOWN);
-                    *abort_flag = 1;
-                    mbar_arrive(&full[s]);   // the phase now completes once the weights have landed
-                    break;
-                }
-                mx_fence_proxy_global();
-                mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ng * (kMxPlaneTile + kMxPlaneScale)));
-                for (int e = 0; e < ng; ++e) {
-                    const uint8_t* pb;
-                    const uint8_t* ps;
-                    if (up) {
-                        const int ent = entry_of(p0 + e);
-                        const size_t tt = ent < 0 ? 0 : static_cast<size_t>(ent / k) * KU + ku;
-                        pb = ent < 0 ? a.zero : a.xp + tt * kMxPlaneTile;
-                        ps = ent < 0 ? a.zero : a.xsf + tt * kMxPlaneScale;
-                    } else {
-                        const size_t tt = static_cast<size_t>(p0 + e) * KD + ku;
-                        pb = a.hp + tt * kMxPlaneTile;
-                        ps = a.hsf + tt * kMxPlaneScale;
+                if (mB < mA) {                         // the B operand of my oldest unit without one
+                    const int i = pw + mB * kMxProducers, s = i % S;
+                    bool up;
+                    int gs, tile, mat, ku;
+                    unit(i, up, gs, tile, mat, ku);
+                    const int slot = act_slot[gs_a[gs]];
+                    bool ready = slot < 0;
+                    if (!ready && up) {
+                        if (!x_ok) x_ok = mx_ld_acquire(x_cnt) >= static_cast<unsigned int>(G);
+                        ready = x_ok;
+                    } else if (!ready) {
+                        if (ready_item != gs * RT + ku && mx_ld_acquire(a.ready + gs * RT + ku) == tag)
+                            ready_item = gs * RT + ku;
+                        ready = ready_item == gs * RT + ku;
                     }
-                    bulk_g2s_nohint(dst + kMxOffB + e * kMxPlaneTile, pb, kMxPlaneTile, &full[s]);
-                    bulk_g2s_nohint(dst + off_sfb + e * kMxPlaneScale, ps, kMxPlaneScale, &full[s]);
+                    if (ready) {
+                        if (slot < 0) {
+                            mbar_arrive(&full[s]);
+                        } else {
+                            const int ng = gs_n[gs], p0 = gs_p0[gs];
+                            uint8_t* dst = ring + static_cast<size_t>(s) * SB;
+                            mx_fence_proxy_global();
+                            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ng * (kMxPlaneTile + kMxPlaneScale)));
+                            for (int e = 0; e < ng; ++e) {
+                                const uint8_t* pb;
+                                const uint8_t* ps;
+                                if (up) {
+                                    const int ent = entry_of(p0 + e);
+                                    const size_t tt = ent < 0 ? 0 : static_cast<size_t>(ent / k) * KU + ku;
+                                    pb = ent < 0 ? a.zero : a.xp + tt * kMxPlaneTile;
+                                    ps = ent < 0 ? a.zero : a.xsf + tt * kMxPlaneScale;
+                                } else {
+                                    const size_t tt = static_cast<size_t>(p0 + e) * KD + ku;
+                                    pb = a.hp + tt * kMxPlaneTile;
+                                    ps = a.hsf + tt * kMxPlaneScale;
+                                }
+                                bulk_g2s_nohint(dst + kMxOffB + e * kMxPlaneTile, pb, kMxPlaneTile, &full[s]);
+                                bulk_g2s_nohint(dst + off_sfb + e * kMxPlaneScale, ps, kMxPlaneScale, &full[s]);
+                            }
+                        }
+                        ++mB;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    t_idle = global_timer_ns();
+                } else {
+                    if (*abort_flag) break;
+                    if (global_timer_ns() - t_idle > a.timeout_ns) {
+                        latch_error(a.err, ERR_ETIMEOUT, 200 + pw, KID_UP);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    __nanosleep(64);
                 }
             }
-            if (*abort_flag) {   // this warp's copies in flight land before the CTA may exit
-                volatile int fresh = 0;
-                for (int j = pw; j < i && j < n_units; j += kMxProducers) {
-                    // a later unit in the same slot was only copied after unit j had been consumed
-                    if (reinterpret_cast<volatile int*>(last_issue)[j % S] != j) continue;
+            if (mB < nm) {   // gave up: the units whose B was never issued complete once their weights land
+                for (int m = mB; m < mA; ++m) mbar_arrive(&full[(pw + m * kMxProducers) % S]);
+                volatile int fresh = 0;   // then every copy of this warp in flight lands before the CTA may exit
+                for (int m = 0; m < mA; ++m) {
+                    const int i = pw + m * kMxProducers;
+                    // a later unit in the same slot was only copied after unit i had been consumed
+                    if (reinterpret_cast<volatile int*>(last_issue)[i % S] != i) continue;
                     fresh = 0;
-                    mbar_wait(&full[j % S], (j / S) & 1, &fresh);
+                    mbar_wait(&full[i % S], (i / S) & 1, &fresh);
                 }
             }
         }
@@ -597,46 +736,53 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
             const uint32_t t_sfa = tmem + 384 + 8 * w, t_sfb = t_sfa + 4;
             const uint32_t w3off = 8 * GM;
             int i = 0;   // CTA-local unit index
+            int j = 0;   // part index
             bool alive = true;
-            for (int j = 0; j < n_parts && alive; ++j) {
+            for (int sg = 0; sg < n_seg && alive; ++sg) {
                 bool up;
-                int item, ua, ub;
-                part_of(j, up, item, ua, ub);
-                const int gs = up ? item / RT : item / NT;
-                const int slot = act_slot[gs_a[gs]];
-                const uint32_t idesc0 = mx_idesc(8 * gs_n[gs], 0), idesc1 = mx_idesc(8 * gs_n[gs], 2);
-                const int db = j & 1;
-                if (j >= 2 && !mbar_poll(&acce[db], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) {
-                    latch_error(a.err, ERR_ETIMEOUT, j, up ? KID_UP : KID_DOWN);
-                    break;
-                }
-                mx_fence_after();
-                bool started0 = false, started1 = false;
-                for (int gu = ua; gu < ub; ++gu, ++i) {
-                    if (i % kMxIssuers != w) continue;
-                    const int s = i % S;
-                    if (!mbar_poll(&full[s], (i / S) & 1, abort_flag, a.timeout_ns)) {
-                        latch_error(a.err, ERR_ETIMEOUT, i, up ? KID_UP : KID_DOWN);
+                int c, base, n, ua, ub;
+                segment(sg, up, c, base, n, ua, ub);
+                if (ua == ub) continue;
+                const int per = up ? upi : dpi;
+                for (int item = ua / per; item <= (ub - 1) / per && alive; ++item, ++j) {
+                    const int pa = max(ua, item * per), pb = min(ub, (item + 1) * per);
+                    const int gs = up ? item / RT : item / NT;
+                    const int slot = act_slot[gs_a[gs]];
+                    const uint32_t idesc0 = mx_idesc(8 * gs_n[gs], 0), idesc1 = mx_idesc(8 * gs_n[gs], 2);
+                    const int db = j & 1;
+                    if (j >= 2 && !mbar_poll(&acce[db], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) {
+                        latch_error(a.err, ERR_ETIMEOUT, j, up ? KID_UP : KID_DOWN);
                         alive = false;
                         break;
                     }
                     mx_fence_after();
-                    if (slot >= 0) {
-                        const int mat = up ? (gu - item * upi) / KU : 0;
-                        const uint32_t dcol = tmem + (db * kMxIssuers + w) * acc_cols + mat * w3off;
-                        const uint32_t sa = ring_base + static_cast<uint32_t>(s) * SB;
-                        mx_cp_atom(t_sfa, sa + kUnitCodeBytes);
-                        mx_cp_atom(t_sfb, sa + off_sfb);
-                        const bool started = mat ? started1 : started0;
-                        mx_mma(dcol, mx_desc(sa, 128, 512), mx_desc(sa + kMxOffB, 128, 512), idesc0, t_sfa, t_sfb,
-                               started ? 1u : 0u);
-                        mx_mma(dcol, mx_desc(sa + 256, 128, 512), mx_desc(sa + kMxOffB + 256, 128, 512), idesc1,
-                               t_sfa | (2u << 30), t_sfb | (2u << 30), 1u);
-                        if (mat) started1 = true; else started0 = true;
+                    bool started0 = false, started1 = false;
+                    for (int gu = pa; gu < pb; ++gu, ++i) {
+                        if (i % kMxIssuers != w) continue;
+                        const int s = i % S;
+                        if (!mbar_poll(&full[s], (i / S) & 1, abort_flag, a.timeout_ns)) {
+                            latch_error(a.err, ERR_ETIMEOUT, i, up ? KID_UP : KID_DOWN);
+                            alive = false;
+                            break;
+                        }
+                        mx_fence_after();
+                        if (slot >= 0) {
+                            const int mat = up ? (gu - item * upi) / KU : 0;
+                            const uint32_t dcol = tmem + (db * kMxIssuers + w) * acc_cols + mat * w3off;
+                            const uint32_t sa = ring_base + static_cast<uint32_t>(s) * SB;
+                            mx_cp_atom(t_sfa, sa + kUnitCodeBytes);
+                            mx_cp_atom(t_sfb, sa + off_sfb);
+                            const bool started = mat ? started1 : started0;
+                            mx_mma(dcol, mx_desc(sa, 128, 512), mx_desc(sa + kMxOffB, 128, 512), idesc0, t_sfa, t_sfb,
+                                   started ? 1u : 0u);
+                            mx_mma(dcol, mx_desc(sa + 256, 128, 512), mx_desc(sa + kMxOffB + 256, 128, 512), idesc1,
+                                   t_sfa | (2u << 30), t_sfb | (2u << 30), 1u);
+                            if (mat) started1 = true; else started0 = true;
+                        }
+                        mx_commit(&empty[s]);   // the slot is free once these MMAs have read it
                     }
-                    mx_commit(&empty[s]);   // the slot is free once these MMAs have read it
+                    if (alive) mx_commit(&accf[db]);   // this issuer's share of the part is done
                 }
-                if (alive) mx_commit(&accf[db]);   // this issuer's share of the part is done
             }
             mx_commit(&fin[w]);              // every MMA of this issuer completes before TMEM is released
             volatile int fresh = 0;
@@ -648,146 +794,186 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
         // ------------------------------------------------------------ epilogue (128 threads, row = thread)
         const uint32_t lane_base = tmem_s + (static_cast<uint32_t>(32 * warp) << 16);
         const int row = 32 * warp + lane;
-        for (int j = 0; j < n_parts; ++j) {
+        int i = 0;   // CTA-local index of the part's first unit
+        int j = 0;   // part index
+        for (int sg = 0; sg < n_seg; ++sg) {
             bool up;
-            int item, ua, ub;
-            part_of(j, up, item, ua, ub);
-            const int gs = up ? item / RT : item / NT, tile = up ? item - gs * RT : item - gs * NT;
-            const int ng = gs_n[gs], p0 = gs_p0[gs], slot = act_slot[gs_a[gs]];
-            const int db = j & 1;
-            // A wait that gives up does not leave the loop: the four warps take the
-            // same named barriers whatever their own waits returned (a warp that
-            // left would strand the others); the outputs of a launch that gave
-            // up are not used, and later waits return at once.
-            int ok = 1;
-            if (lane == 0) ok = mbar_poll(&accf[db], (j >> 1) & 1, abort_flag, a.timeout_ns);
-            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-            if (!ok && lane == 0) latch_error(a.err, ERR_ETIMEOUT, j, up ? KID_UP : KID_DOWN);
-            mx_fence_after();
-            const int per = up ? upi : dpi, nall = up ? NU : ND;
-            const int ibase = item * per;
-            // units of w1 (or w2) and of w3 in this part, and the CTA-local index of the part's first unit
-            const int m0a = ua, m0b = up ? min(ub, ibase + KU) : ub;
-            const int m1a = up ? max(ua, ibase + KU) : ub, m1b = ub;
-            const int i0 = up ? ua - u0 : nu + (ua - d0);
-            float acc0[kMxGroup], acc1[kMxGroup];
-#pragma unroll
-            for (int e = 0; e < kMxGroup; ++e) {
-                acc0[e] = 0.0f;
-                acc1[e] = 0.0f;
-            }
-            for (int w = 0; w < kMxIssuers; ++w) {   // fixed order: results do not depend on timing
-                // issuer w took unit gu iff (i0 + gu - ua) % kMxIssuers == w
-                const int f0 = m0a + ((w - (i0 + m0a - ua)) % kMxIssuers + kMxIssuers) % kMxIssuers;
-                const int f1 = m1a + ((w - (i0 + m1a - ua)) % kMxIssuers + kMxIssuers) % kMxIssuers;
-                const bool t0 = f0 < m0b, t1 = f1 < m1b;
-                const uint32_t dw = lane_base + (db * kMxIssuers + w) * acc_cols;
-#pragma unroll
-                for (int e = 0; e < kMxGroup; ++e) {
-                    if (ok && slot >= 0 && e < ng) {
-                        if (t0) acc0[e] += mx_ld8_sum(dw + 8 * e);
-                        if (t1) acc1[e] += mx_ld8_sum(dw + 8 * GM + 8 * e);
-                    }
-                }
-            }
-            mx_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[db]);   // the MMAs may reuse this accumulator
-            // the CTAs holding units of this item, in order
-            const int bf = mx_cta_of(nall, G, ibase), bl = mx_cta_of(nall, G, ibase + per - 1);
-            int nparts = 0;
-            for (int bb = bf; bb <= bl; ++bb)
-                nparts += mx_range_start(nall, G, bb) < mx_range_start(nall, G, bb + 1);
-            if (nparts > 1) {   // split item: store this part, the last part to arrive adds them all
-                const int side = (item == (up ? up_first : dn_first)) ? 0 : 1;
-                float* pp = a.part + static_cast<size_t>(b) * kMxPartFloats +
-                            (up ? side * kMxPartUp : 2 * kMxPartUp + side * kMxPartDown);
-#pragma unroll
-                for (int e = 0; e < kMxGroup; ++e) {
-                    if (e < ng) {
-                        pp[e * 128 + row] = acc0[e];
-                        if (up) pp[kMxGroup * 128 + e * 128 + row] = acc1[e];
-                    }
-                }
-                mx_named_barrier(1, kMxEpiWarps * 32);
-                if (tid == 0) {
-                    __threadfence();
-                    const unsigned int c = mx_arrive(up ? up_cnt + item : dn_cnt + item);
-                    last_s = c == static_cast<unsigned int>(nparts);
-                }
-                mx_named_barrier(1, kMxEpiWarps * 32);
-                if (!last_s) continue;
-                __threadfence();
+            int c, base, n, ua, ub;
+            segment(sg, up, c, base, n, ua, ub);
+            if (ua == ub) continue;
+            const int per = up ? upi : dpi;
+            const int first_item = ua / per;
+            for (int item = first_item; item <= (ub - 1) / per; ++item, ++j) {
+                const int pa = max(ua, item * per), pb = min(ub, (item + 1) * per);
+                const int i0 = i;
+                i += pb - pa;
+                const int gs = up ? item / RT : item / NT, tile = up ? item - gs * RT : item - gs * NT;
+                const int ng = gs_n[gs], p0 = gs_p0[gs], slot = act_slot[gs_a[gs]];
+                const int db = j & 1;
+                // A wait that gives up does not leave the loop: the four warps take the
+                // same named barriers whatever their own waits returned (a warp that
+                // left would strand the others); the outputs of a launch that gave
+                // up are not used, and later waits return at once.
+                int ok = 1;
+                if (lane == 0) ok = mbar_poll(&accf[db], (j >> 1) & 1, abort_flag, a.timeout_ns);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok && lane == 0) latch_error(a.err, ERR_ETIMEOUT, j, up ? KID_UP : KID_DOWN);
+                mx_fence_after();
+                const int ibase = item * per;
+                // units of w1 (or w2) and of w3 in this part
+                const int m0a = pa, m0b = up ? min(pb, ibase + KU) : pb;
+                const int m1a = up ? max(pa, ibase + KU) : pb, m1b = pb;
+                float acc0[kMxGroup], acc1[kMxGroup];
 #pragma unroll
                 for (int e = 0; e < kMxGroup; ++e) {
                     acc0[e] = 0.0f;
                     acc1[e] = 0.0f;
                 }
-                for (int bb = bf; bb <= bl; ++bb) {
-                    const int st = mx_range_start(nall, G, bb);
-                    if (st == mx_range_start(nall, G, bb + 1)) continue;
-                    const int sd = (item == st / per) ? 0 : 1;
-                    const float* q = a.part + static_cast<size_t>(bb) * kMxPartFloats +
-                                     (up ? sd * kMxPartUp : 2 * kMxPartUp + sd * kMxPartDown);
+                const int ncols = up ? 16 * GM : 8 * GM;   // this part's columns of one issuer
+                // issuer w took unit gu iff (i0 + gu - pa) % kMxIssuers == w; did it reach w1 (w2) / w3 units?
+                auto touched = [&](int w, bool& t0, bool& t1) {
+                    const int f0 = m0a + ((w - (i0 + m0a - pa)) % kMxIssuers + kMxIssuers) % kMxIssuers;
+                    const int f1 = m1a + ((w - (i0 + m1a - pa)) % kMxIssuers + kMxIssuers) % kMxIssuers;
+                    t0 = f0 < m0b;
+                    t1 = f1 < m1b;
+                };
+                // sums of one issuer's columns: w1 (w2) planes at 8 e, w3 planes at 8 GM + 8 e
+                auto add = [&](const uint32_t* r, bool t0, bool t1) {
 #pragma unroll
                     for (int e = 0; e < kMxGroup; ++e) {
                         if (e < ng) {
-                            acc0[e] += __ldcg(q + e * 128 + row);
-                            if (up) acc1[e] += __ldcg(q + kMxGroup * 128 + e * 128 + row);
+                            float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                s0 += __uint_as_float(r[8 * e + q]);
+                                s1 += __uint_as_float(GM == 1 ? r[(8 + 8 * e + q) & 31] : r[(16 + 8 * e + q) & 31]);
+                            }
+                            if (t0) acc0[e] += s0;
+                            if (t1) acc1[e] += s1;
+                        }
+                    }
+                };
+                if (ok && slot >= 0) {
+                    if (ncols <= 16) {   // two issuers per TMEM round trip, fixed order
+                        for (int w = 0; w < kMxIssuers; w += 2) {
+                            bool ta0, ta1, tb0, tb1;
+                            touched(w, ta0, ta1);
+                            touched(w + 1, tb0, tb1);
+                            uint32_t ra[16], rb[16];
+                            if (ta0 || ta1) mx_ld_issue16(lane_base + (db * kMxIssuers + w) * acc_cols, ncols, ra);
+                            if (tb0 || tb1) mx_ld_issue16(lane_base + (db * kMxIssuers + w + 1) * acc_cols, ncols, rb);
+                            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                            if (ta0 || ta1) add(ra, ta0, ta1);
+                            if (tb0 || tb1) add(rb, tb0, tb1);
+                        }
+                    } else {
+                        for (int w = 0; w < kMxIssuers; ++w) {
+                            bool t0, t1;
+                            touched(w, t0, t1);
+                            if (!(t0 || t1)) continue;
+                            uint32_t r[32];
+                            mx_ld_cols(lane_base + (db * kMxIssuers + w) * acc_cols, ncols, r);
+                            add(r, t0, t1);
                         }
                     }
                 }
-            }
-            if (up) {
-                // h = bf16(silu(a1) * a3) of rows 128 tile + row, then its digit planes (block = warp)
+                mx_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[db]);   // the MMAs may reuse this accumulator
+                // the CTAs holding units of this up item (relative to the chunk's unit space), in order;
+                // a down item is never cut
+                const int bf = up ? mx_cta_of(n, G, ibase - base) : b;
+                const int bl = up ? mx_cta_of(n, G, ibase - base + per - 1) : b;
+                int nparts = up ? 0 : 1;
+                for (int bb = bf; up && bb <= bl; ++bb) nparts += mx_range_start(n, G, bb) < mx_range_start(n, G, bb + 1);
+                if (nparts > 1) {   // split item: store this part, the last part to arrive adds them all
+                    const int side = (item == first_item) ? 0 : 1;
+                    float* pp = a.part + static_cast<size_t>(b) * kMxPartFloats + c * kMxPartChunk +
+                                (up ? side * kMxPartUp : 2 * kMxPartUp + side * kMxPartDown);
 #pragma unroll
-                for (int e = 0; e < kMxGroup; ++e) {
-                    if (e < ng) {
-                        const float a1 = acc0[e], a3 = acc1[e];
-                        const float hv = (slot >= 0) ? a1 / (1.0f + expf(-a1)) * a3 : 0.0f;
-                        const float hf = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rne(hv)) << 16);
-                        const size_t tt = static_cast<size_t>(p0 + e) * KD + tile;
-                        mx_split_block(hf, lane, a.hp + tt * kMxPlaneTile + warp * 128, a.hsf + tt * kMxPlaneScale + warp);
+                    for (int e = 0; e < kMxGroup; ++e) {
+                        if (e < ng) {
+                            pp[e * 128 + row] = acc0[e];
+                            if (up) pp[kMxGroup * 128 + e * 128 + row] = acc1[e];
+                        }
                     }
-                }
-                mx_named_barrier(1, kMxEpiWarps * 32);
-                if (tid == 0) {
+                    mx_named_barrier(1, kMxEpiWarps * 32);
+                    if (tid == 0) {   // the acquire-release add orders the CTA's stores (named barrier) before it
+                        const unsigned int cnt = mx_arrive(up ? up_cnt + item : dn_cnt + item);
+                        last_s = cnt == static_cast<unsigned int>(nparts);
+                    }
+                    mx_named_barrier(1, kMxEpiWarps * 32);
+                    if (!last_s) continue;
                     __threadfence();
-                    mx_fence_proxy_global();
-                    mx_st_release(a.ready + item, tag);
-                    if (slot < 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gs]], KID_UP);
-                }
-            } else {
 #pragma unroll
-                for (int e = 0; e < kMxGroup; ++e) {
-                    if (e < ng) {
-                        const int ent = entry_of(p0 + e);
-                        if (ent >= 0)
-                            a.obuf[static_cast<size_t>(ent) * H + tile * 128 + row] = (slot >= 0) ? acc0[e] : 0.0f;
+                    for (int e = 0; e < kMxGroup; ++e) {
+                        acc0[e] = 0.0f;
+                        acc1[e] = 0.0f;
+                    }
+                    for (int bb = bf; bb <= bl; ++bb) {
+                        const int st = mx_range_start(n, G, bb);
+                        if (st == mx_range_start(n, G, bb + 1)) continue;
+                        const int sd = (item == (base + st) / per) ? 0 : 1;
+                        const float* q = a.part + static_cast<size_t>(bb) * kMxPartFloats + c * kMxPartChunk +
+                                         (up ? sd * kMxPartUp : 2 * kMxPartUp + sd * kMxPartDown);
+#pragma unroll
+                        for (int e = 0; e < kMxGroup; ++e) {
+                            if (e < ng) {
+                                acc0[e] += __ldcg(q + e * 128 + row);
+                                if (up) acc1[e] += __ldcg(q + kMxGroup * 128 + e * 128 + row);
+                            }
+                        }
                     }
                 }
-                if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gs]], KID_DOWN);
-                if (a.y != nullptr) {
-                    // the CTA finishing the last item of this 128-row tile combines it for every token
-                    mx_named_barrier(1, kMxEpiWarps * 32);
-                    if (tid == 0) {
-                        __threadfence();
-                        last_s = mx_arrive(tile_cnt + tile) == static_cast<unsigned int>(n_gs);
+                if (up) {
+                    // h = bf16(silu(a1) * a3) of rows 128 tile + row, then its digit planes (block = warp)
+#pragma unroll
+                    for (int e = 0; e < kMxGroup; ++e) {
+                        if (e < ng) {
+                            const float a1 = acc0[e], a3 = acc1[e];
+                            const float hv = (slot >= 0) ? a1 / (1.0f + expf(-a1)) * a3 : 0.0f;
+                            const float hf = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rne(hv)) << 16);
+                            const size_t tt = static_cast<size_t>(p0 + e) * KD + tile;
+                            mx_split_block(hf, lane, a.hp + tt * kMxPlaneTile + warp * 128,
+                                           a.hsf + tt * kMxPlaneScale + warp);
+                        }
                     }
                     mx_named_barrier(1, kMxEpiWarps * 32);
-                    if (last_s) {
-                        __threadfence();
-                        const int n0 = tile * 128 + row;
-                        for (int t = 0; t < a.T; ++t) {
-                            float yv = 0.0f;
-                            for (int jj = 0; jj < k; ++jj) {
-                                const float wj = routed ? r_w[t * k + jj] : __ldg(a.weights + t * k + jj);
-                                yv = fmaf(wj, __ldcg(a.obuf + static_cast<size_t>(t * k + jj) * H + n0), yv);
-                            }
-                            a.y[static_cast<size_t>(t) * H + n0] = yv;
-                            if (a.x_out) {
-                                const float xv = bf16_to_f32(a.x[static_cast<size_t>(t) * H + n0]);
-                                a.x_out[static_cast<size_t>(t) * H + n0] = f32_to_bf16_rne(xv + yv);
+                    if (tid == 0) {   // the release store orders the CTA's stores (named barrier) before it
+                        mx_fence_proxy_global();
+                        mx_st_release(a.ready + item, tag);
+                        if (slot < 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gs]], KID_UP);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kMxGroup; ++e) {
+                        if (e < ng) {
+                            const int ent = entry_of(p0 + e);
+                            if (ent >= 0)
+                                a.obuf[static_cast<size_t>(ent) * H + tile * 128 + row] = (slot >= 0) ? acc0[e] : 0.0f;
+                        }
+                    }
+                    if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[gs_a[gs]], KID_DOWN);
+                    if (a.y != nullptr) {
+                        // the CTA finishing the last item of this 128-row tile combines it for every token
+                        mx_named_barrier(1, kMxEpiWarps * 32);
+                        if (tid == 0)
+                            last_s = mx_arrive(tile_cnt + tile) == static_cast<unsigned int>(n_gs);
+                        mx_named_barrier(1, kMxEpiWarps * 32);
+                        if (last_s) {
+                            __threadfence();
+                            const int n0 = tile * 128 + row;
+                            for (int t = 0; t < a.T; ++t) {
+                                float yv = 0.0f;
+                                for (int jj = 0; jj < k; ++jj) {
+                                    const float wj = routed ? r_w[t * k + jj] : __ldg(a.weights + t * k + jj);
+                                    yv = fmaf(wj, __ldcg(a.obuf + static_cast<size_t>(t * k + jj) * H + n0), yv);
+                                }
+                                a.y[static_cast<size_t>(t) * H + n0] = yv;
+                                if (a.x_out) {
+                                    const float xv = bf16_to_f32(a.x[static_cast<size_t>(t) * H + n0]);
+                                    a.x_out[static_cast<size_t>(t) * H + n0] = f32_to_bf16_rne(xv + yv);
+                                }
                             }
                         }
                     }
