@@ -121,7 +121,8 @@ __device__ void group_entries(const RouteArgs& a, int* hist) {
     for (int b = lo; b < hi; b += 32) {
         int i = b + lane;
         int e = (i < hi) ? ld_cg(a.ids + i) : -1;
-        if (e >= E || (i < hi && e < 0)) { latch_error(a.err, ERR_EINVAL, i, KID_ROUTE); e = -1; }
+        // id -1 marks an empty entry (left out silently); any other id outside [0, E) is an error
+        if (e >= E || e < -1) { latch_error(a.err, ERR_EINVAL, i, KID_ROUTE); e = -1; }
         uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
     }

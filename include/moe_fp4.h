@@ -272,8 +272,10 @@ moe_fp4_status moe_fp4_route_forward(moe_fp4_ctx *ctx, int layer, const float *l
  * processes (token, slot) entries, so listing a forward's entries in
  * (token, slot) order reproduces its per-entry outputs bit for bit.
  *  x        bf16 [n, H] device, 16-byte aligned (row i goes with experts[i]).
- *  experts  int32 [n] device; an id outside [0, E) latches EINVAL and its
- *           row of o is left unwritten.
+ *  experts  int32 [n] device; id -1 marks an empty entry (no work, its row
+ *           of o is left unwritten: the expert-parallel exchange pads with
+ *           it); any other id outside [0, E) latches EINVAL and its row of o
+ *           is left unwritten.
  *  o        fp32 [n, H] device out, 16-byte aligned.
  * n <= max_tokens * top_k; uses the context's workspace like forward.
  * Errors: EINVAL, ECUDA; unmapped experts latch ESLOT (their rows are zero).

@@ -47,3 +47,13 @@ def test_drafter_batch256(drafter, path):
     rng = np.random.default_rng(5)
     toks = sorted({int(np.nonzero((ids == hot).any(1))[0][-1]), 255, *map(int, rng.choice(256, 5, replace=False))})
     check_y(y[toks], drafter.oracle_y(0, x, ids, w, toks))
+
+
+def test_drafter_batch256_paths_agree_on_every_token(drafter):
+    """The decode kernel (groups of two entries, 768 entries) and the tcgen05 path
+    on the same 256-token batch: every token within twice the bar of each other
+    (both are within the bar of the oracle on the sampled tokens above)."""
+    wl = synth.WORKLOADS["drafter_b256"]
+    ys = {path: _run(drafter, wl, 256, 3, path)[3] for path in (moe.PATH_GEMV, moe.PATH_TC)}
+    drafter.ctx.set_path(moe.PATH_AUTO)
+    check_y(ys[moe.PATH_GEMV], ys[moe.PATH_TC].astype(np.float64), tol=2e-2)

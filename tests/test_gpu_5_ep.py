@@ -1,7 +1,8 @@
 """The expert-parallel building blocks on the GPU: moe_fp4_expert_outputs on
 a forward's (token, slot) entries followed by moe_fp4_combine must reproduce
 moe_fp4_forward bit for bit (same per-expert grouping, same kernels), and the
-expert-parallel driver over a one-rank NCCL group must give the same y."""
+expert-parallel driver over a one-rank NCCL group, with either dispatch plan,
+must give the same y and meet the oracle bar on every token."""
 import os
 import socket
 
@@ -11,7 +12,7 @@ import torch
 import torch.distributed as dist
 
 from fp4_routed_expert_router_b200 import ep, moe, synth
-from tests.gpu_helpers import Filled, to_dev
+from tests.gpu_helpers import Filled, check_y, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +58,11 @@ def test_v41_expert_outputs_and_combine_equal_forward(v41, path):
     _pieces_vs_forward(v41, 64, 4100, path)
 
 
-def test_expert_parallel_driver_one_rank_nccl(tiny):
+@pytest.mark.parametrize("device_plan", [True, False])
+def test_expert_parallel_driver_one_rank_nccl(tiny, device_plan):
+    """The driver over a one-rank NCCL group, with the device plan (fixed-capacity
+    slots padded with expert id -1, no host read) or the host plan: y equals
+    moe_fp4_forward bit for bit and meets the oracle bar on every token."""
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
@@ -66,10 +71,17 @@ def test_expert_parallel_driver_one_rank_nccl(tiny):
     dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
                             device_id=torch.device("cuda", 0))
     try:
-        r, xd, y = _pieces_vs_forward(tiny, 33, 4200, moe.PATH_AUTO)
-        layer = ep.ExpertParallel(tiny.wl.n_experts, tiny.wl.top_k, tiny.wl.hidden)
-        y_ep = layer.forward(xd, r.ids, r.weights, ep.gpu_expert_fn(tiny.ctx, 0), ep.gpu_combine_fn(tiny.ctx))
+        T, step = 33, 4200
+        r, xd, y = _pieces_vs_forward(tiny, T, step, moe.PATH_AUTO)
+        wl = tiny.wl
+        layer = ep.ExpertParallel(wl.n_experts, wl.top_k, wl.hidden, max_tokens=48)
+        y_ep = layer.forward(xd, r.ids, r.weights, ep.gpu_expert_fn(tiny.ctx, 0), ep.gpu_combine_fn(tiny.ctx),
+                             device_plan=device_plan)
         torch.cuda.synchronize()
+        rc, msg = tiny.ctx.last_error()
+        assert rc == moe.OK, msg
         assert torch.equal(y_ep, y)
+        x = synth.gen_x(wl.seed, T, wl.hidden, step)
+        check_y(y_ep.cpu().numpy(), tiny.oracle_y(0, x, r.ids.cpu().numpy(), r.weights.cpu().numpy(), range(T)))
     finally:
         dist.destroy_process_group()
