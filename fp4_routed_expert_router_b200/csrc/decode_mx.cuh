@@ -28,29 +28,36 @@
 //
 // Work.  A unit is one 128-row x 128-K tile of one weight matrix (8,704
 // bytes: codes and block scales, slot_layout.cuh) plus the B tile of its
-// token group (<= 4 entries x 8 planes x 128 K, and their scale bytes).  An
-// up item is (token group, 128 rows of w1 and w3) over all of H; a down item
-// (group, 128 rows of w2) over all of I.  The up units of all items form one
-// sequence split contiguously over the CTAs (one per SM), the down units
-// another; an item cut by a range boundary is finished by whichever of its
-// CTAs completes last, which adds the fp32 partials in CTA order (results do
-// not depend on timing).  Inside a CTA:
+// token group (<= 2 entries x 8 planes x 128 K, and their scale bytes; one
+// entry per group for a single token).  An up item is (token group, 128 rows
+// of w1 and w3) over all of H; a down item (group, 128 rows of w2) over all
+// of I.  The up units of all items form one sequence split contiguously over
+// the CTAs (one per SM); an up item cut by a range boundary is finished by
+// whichever of its CTAs completes last, which adds the fp32 partials in CTA
+// order (results do not depend on timing).  Down items are dealt out whole,
+// so no down partial crosses CTAs.  Inside a CTA:
 //   warps 10-15         producers, one lane per ring slot (S / 6 lanes each):
 //                       bulk copies of unit i (A + scales from the arena, B +
-//                       B scales from the plane buffers) into slot i % S;
-//   warps 4-6, lane 0   MMA issuers: issuer i % 3 takes unit i -- tcgen05.cp
-//                       of both scale atoms into its own TMEM columns, two
-//                       K = 64 MMAs into its own double-buffered accumulator,
-//                       tcgen05.commit frees the slot.  One thread's tcgen05
-//                       stream stalls at every commit (measured on B200: one
-//                       issuer 307 ns per unit, three keep the pipe ahead of
-//                       HBM), so three issuers take turns;
+//                       B scales from the plane buffers) into slot i % S.  A
+//                       lane copies the weights as soon as its slot is free
+//                       and the B tile once it exists, so weights stream
+//                       ahead of the activations they meet;
+//   warps 4-9, lane 0   MMA issuers: slot s belongs to issuer s % 6 --
+//                       tcgen05.cp of both scale atoms into its own TMEM
+//                       columns, two K = 64 MMAs into its own double-buffered
+//                       accumulator, tcgen05.commit frees the slot.  One
+//                       thread's tcgen05 stream stalls at every commit
+//                       (measured on B200: one issuer 307 ns per unit, two
+//                       154, four 77), so six issuers take turns and keep the
+//                       pipe ahead of HBM;
 //   warps 0-3           epilogue (TMEM lane quadrant = warp): planes and the
-//                       issuers' accumulators summed (fixed order), then a partial, or the item's finish: SwiGLU, bf16 h
-//                       and its digit planes (up), per-entry o and the
-//                       combine of a 128-row output tile by the CTA that
-//                       completes its last item (down);
-//   all warps           prologue: routing, and a share of the x planes.
+//                       issuers' accumulators summed (fixed order), then a
+//                       partial, or the item's finish: SwiGLU, bf16 h and its
+//                       digit planes (up), per-entry o and the combine of a
+//                       128-row output tile by the CTA that completes its
+//                       last item (down);
+//   all warps           prologue: routing, and a share of the x planes; the
+//                       mbarrier and TMEM set-up runs in warp 4 meanwhile.
 // Ordering across CTAs has no grid barrier: the x planes are counted, every
 // up item raises a flag once its h planes are stored, and a producer lane
 // checks the flag (acquire) before it copies the h planes of a down unit --

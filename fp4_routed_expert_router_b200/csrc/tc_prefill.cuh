@@ -34,10 +34,11 @@
 //                gathered token rows (x grouped by expert, or h, both as f16
 //                with an exact power-of-two prescale per row), 128-byte
 //                swizzle, into shared memory.
-//   warp 21      code producer: cp.async.bulk of the item's rows of one
-//                128-K unit per stage (up: rows 64h.. of the w1 and the w3
-//                unit and both scale atoms; down: the whole w2 unit) into a
-//                ring.
+//   warp 21      code producer: cp.async.bulk of the item's rows of two
+//                128-K units (one when K / 128 is odd) per ring entry (up:
+//                rows 64h.. of the w1 and the w3 unit and both scale atoms;
+//                down: the whole w2 unit); the dequantisers free an entry
+//                once, after both of its stages.
 //   warp 22      MMA issuer: tcgen05.mma.cta_group::1.kind::f16 (f16 x f16)
 //                with A from TMEM and B from shared memory (fp32 accumulate
 //                in TMEM), eight
@@ -82,7 +83,8 @@ struct TcArgs {
     int T;
     int off_b;             // dynamic smem offset of the B ring (1024-aligned), kTcStages x 2 atoms x kTcNmax rows x 128 bytes
     int off_code;          // offset of the code ring: centries x entry_bytes
-    int entry_bytes;       // the item's slot blocks for one block's K (4 up / 8 down blocks)
+    int entry_bytes;       // one code ring entry: spe units' worth of the item's rows
+    int spe;               // 128-K units (= stages) per code entry: 2 when K / 128 is even, else 1
     int centries;          // 0 when the shape does not fit
     int max_active;
     unsigned long long timeout_ns;   // limit of each bounded wait
@@ -240,8 +242,10 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     const int E = a.E;
     const int K = UP ? a.H : a.I;
     const int n_mt = (UP ? a.I : a.H) / OUT_ROWS;
-    const int nfb = K / kTcSK;                   // code entries (= stages) per item: one 128-K unit each
-    const int n_stg = nfb;
+    const int n_stg = K / kTcSK;                 // stages per item: one 128-K unit each
+    const int spe = t.spe;                       // stages per code entry
+    const int nfb = n_stg / spe;                 // code entries per item
+    const int ustride = t.entry_bytes / spe;     // bytes of one unit inside an entry
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -347,14 +351,15 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
         // up: lanes 0-15 w1 rows, 16-31 w3 rows of the item's 64; down: row 32 lg + lane
         const int mat = UP ? (lane >> 4) : 0;
         const int rloc = UP ? 16 * lg + (lane & 15) : 32 * lg + lane;
-        int gstg = 0;
+        int gstg = 0, gent = 0;
         for (int i = 0; i < my_items; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int slot = act_slot[ai];
             if (slot < 0 && tid == 0) latch_error(a.err, ERR_ESLOT, act_e[ai], kid);
-            // entry layout: up  [w1 rows 64h.. codes 4096][w3 codes 4096][w1 scale atom][w3 scale atom]
-            //               down [the unit, 8704]
+            // entry layout, per unit j at j * ustride:
+            //   up   [w1 rows 64h.. codes 4096][w3 codes 4096][w1 scale atom][w3 scale atom]
+            //   down [the unit, 8704]
             const int urow = UP ? 64 * (mt & 1) + rloc : rloc;       // row inside the 128-row unit
             const int code_off = UP ? mat * 4096 + unit_code_chunk(rloc, cc) : unit_code_chunk(rloc, cc);
             const int scale_off = UP ? 2 * 4096 + mat * kUnitScaleBytes + unit_scale_byte(urow, cc) - kUnitCodeBytes
@@ -364,32 +369,33 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             const int sref = slot < 0 ? 0
                                       : __ldg(t.rowref + static_cast<size_t>(slot) * (2 * a.I + a.H) +
                                               (UP ? mat * a.I : 2 * a.I) + wrow);
-            for (int f = 0; f < nfb; ++f, ++gstg) {
-                const int ce = gstg % CE;
-                if (!mbar_wait(&cfull[ce], (gstg / CE) & 1, abort_flag, t.timeout_ns) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+            for (int f = 0; f < nfb; ++f, ++gent) {
+                const int ce = gent % CE;
+                if (!mbar_wait(&cfull[ce], (gent / CE) & 1, abort_flag, t.timeout_ns) && lane == 0)
+                    latch_error(a.err, ERR_ETIMEOUT, gent, kid);
                 const uint8_t* ent = code_entry(ce);
-                const int st = gstg % S;
-                if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
-                    latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
-                tc_fence_after();
-                const uint4 w = *reinterpret_cast<const uint4*>(ent + code_off);
-                const int sq = ent[scale_off];
-                const uint32_t mult = (slot < 0) ? 0u : mtab[(sref - sq) & 255];
-                uint32_t o[16];
-                e2m1x8_to_f16x2(w.x, o);
-                e2m1x8_to_f16x2(w.y, o + 4);
-                e2m1x8_to_f16x2(w.z, o + 8);
-                e2m1x8_to_f16x2(w.w, o + 12);
+                for (int j = 0; j < spe; ++j, ++gstg) {
+                    const int st = gstg % S;
+                    if (gstg >= S && !mbar_wait(&sfree[st], ((gstg / S) - 1) & 1, abort_flag, t.timeout_ns) &&
+                        lane == 0)
+                        latch_error(a.err, ERR_ETIMEOUT, gstg, kid);
+                    tc_fence_after();
+                    const uint4 w = *reinterpret_cast<const uint4*>(ent + j * ustride + code_off);
+                    const int sq = ent[j * ustride + scale_off];
+                    const uint32_t mult = (slot < 0) ? 0u : mtab[(sref - sq) & 255];
+                    uint32_t o[16];
+                    e2m1x8_to_f16x2(w.x, o);
+                    e2m1x8_to_f16x2(w.y, o + 4);
+                    e2m1x8_to_f16x2(w.z, o + 8);
+                    e2m1x8_to_f16x2(w.w, o + 12);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) o[q] = hmul2_u32(o[q], mult);
-                tmem_st16(tmem_a + lane_addr + st * ACOLS + 16 * cc, o);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&full[st]);
-                    mbar_arrive(&cfree[ce]);
+                    for (int q = 0; q < 16; ++q) o[q] = hmul2_u32(o[q], mult);
+                    tmem_st16(tmem_a + lane_addr + st * ACOLS + 16 * cc, o);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[st]);
                 }
+                if (lane == 0) mbar_arrive(&cfree[ce]);
             }
         }
     } else if (warp < kTcDequantWarps + kTcEpiWarps) {
@@ -509,20 +515,25 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                 if (lane == 0) {
                     if (slot < 0) {
                         mbar_arrive(&cfull[ce]);
-                    } else if (UP) {   // rows 64h .. 64h+63 of the w1 and w3 units (rt, f), and both scale atoms
-                        const int rt = mt >> 1, hh = mt & 1;
-                        const uint8_t* u1 = src + up_unit_offset(L, 0, rt, f);
-                        const uint8_t* u3 = src + up_unit_offset(L, 1, rt, f);
-                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(t.entry_bytes));
-                        bulk_g2s(code_entry(ce), u1 + 4096 * hh, 4096u, &cfull[ce], pol);
-                        bulk_g2s(code_entry(ce) + 4096, u3 + 4096 * hh, 4096u, &cfull[ce], pol);
-                        bulk_g2s(code_entry(ce) + 8192, u1 + kUnitCodeBytes, kUnitScaleBytes, &cfull[ce], pol);
-                        bulk_g2s(code_entry(ce) + 8192 + kUnitScaleBytes, u3 + kUnitCodeBytes, kUnitScaleBytes,
-                                 &cfull[ce], pol);
                     } else {
-                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(kUnitBytes));
-                        bulk_g2s(code_entry(ce), src + down_unit_offset(L, mt, f) - L.up_bytes, kUnitBytes,
-                                 &cfull[ce], pol);
+                        mbar_arrive_expect_tx(&cfull[ce], static_cast<uint32_t>(t.entry_bytes));
+                        for (int j = 0; j < spe; ++j) {
+                            uint8_t* dst = code_entry(ce) + j * ustride;
+                            const int ku = f * spe + j;
+                            if (UP) {   // rows 64h .. 64h+63 of the w1 and w3 units (rt, ku), and both scale atoms
+                                const int rt = mt >> 1, hh = mt & 1;
+                                const uint8_t* u1 = src + up_unit_offset(L, 0, rt, ku);
+                                const uint8_t* u3 = src + up_unit_offset(L, 1, rt, ku);
+                                bulk_g2s(dst, u1 + 4096 * hh, 4096u, &cfull[ce], pol);
+                                bulk_g2s(dst + 4096, u3 + 4096 * hh, 4096u, &cfull[ce], pol);
+                                bulk_g2s(dst + 8192, u1 + kUnitCodeBytes, kUnitScaleBytes, &cfull[ce], pol);
+                                bulk_g2s(dst + 8192 + kUnitScaleBytes, u3 + kUnitCodeBytes, kUnitScaleBytes,
+                                         &cfull[ce], pol);
+                            } else {
+                                bulk_g2s(dst, src + down_unit_offset(L, mt, ku) - L.up_bytes, kUnitBytes,
+                                         &cfull[ce], pol);
+                            }
+                        }
                     }
                 }
                 __syncwarp();
@@ -674,10 +685,11 @@ inline TcArgs tc_args(const TcPlan& p, const ExpertArgs& g, const SlotLayout& L,
     const int head = 1024 + 256 * 16 + 4 * (5 * t.max_active + 1 + 2 * g.E + 1);
     t.off_b = (head + 1023) / 1024 * 1024;
     t.off_code = t.off_b + kTcStages * 2 * kTcNmax * 128;
-    t.entry_bytes = up ? 2 * (4096 + kUnitScaleBytes) : kUnitBytes;
+    const int K = up ? g.H : g.I, rows = up ? g.I : g.H;
+    t.spe = (K / kTcSK) % 2 == 0 ? 2 : 1;
+    t.entry_bytes = t.spe * (up ? 2 * (4096 + kUnitScaleBytes) : kUnitBytes);
     int ce = (p.smem_limit - 1024 - t.off_code) / t.entry_bytes;
     if (ce > kTcMaxEntries) ce = kTcMaxEntries;
-    const int K = up ? g.H : g.I, rows = up ? g.I : g.H;
     const bool shape_ok = (K % kTcSK == 0) && (rows % kTcM == 0);
     t.centries = (ce >= 2 && shape_ok) ? ce : 0;
     return t;
