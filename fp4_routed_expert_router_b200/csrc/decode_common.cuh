@@ -80,17 +80,19 @@ __global__ void __launch_bounds__(256) entry_norm_kernel(const float* obuf, int 
 }
 
 // saliency[e] += sum over e's grouped entries of w * norm, in perm order, fp64.
+// Offsets or entries outside [0, n_ent) (not a grouping of this batch) add nothing.
 __global__ void __launch_bounds__(128) saliency_kernel(const float* norms, const float* w, const int32_t* offsets,
-                                                       const int32_t* perm, int E, double* sal) {
+                                                       const int32_t* perm, int E, int n_ent, double* sal) {
     pdl_wait();
     pdl_trigger();
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     const int p0 = __ldg(offsets + e), p1 = __ldg(offsets + e + 1);
-    if (p1 <= p0) return;
+    if (p1 <= p0 || p0 < 0 || p1 > n_ent) return;
     double acc = 0.0;
     for (int p = p0; p < p1; ++p) {
         const int ent = __ldg(perm + p);
+        if (ent < 0 || ent >= n_ent) continue;
         acc += static_cast<double>(__ldg(w + ent)) * static_cast<double>(norms[ent]);
     }
     sal[e] += acc;

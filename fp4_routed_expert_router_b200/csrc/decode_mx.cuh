@@ -289,27 +289,33 @@ __device__ __forceinline__ void mx_split_block(float v, int lane, uint8_t* pc, u
             e0 = (field - 127) - (frac == 0u ? 1 : 0);
         }
     }
+    // this lane's digit of every plane, one nibble each (plane p in bits 4p .. 4p+3)
     float r = v;
+    uint32_t x = 0u;
 #pragma unroll
     for (int p = 0; p < kMxPlanes; ++p) {
         const int s = e0 - 2 * p;               // plane scale 2^s
-        uint32_t code = 0u;
-        int sbyte = 0;
         if (live && s >= -127) {
             const float d = rintf(2.0f * mx_mul_pow2(r, -s)) * 0.5f;   // nearest half: |d| <= 2
             const float ad = fabsf(d);
-            code = static_cast<uint32_t>(2.0f * ad) | (d < 0.0f ? 8u : 0u);
+            x |= (static_cast<uint32_t>(2.0f * ad) | (d < 0.0f ? 8u : 0u)) << (4 * p);
             r -= mx_mul_pow2(d, s);             // exact: |r| shrinks below 2^(s-2)
-            sbyte = s + 127;
-        } else if (!live && p == 0 && mb != 0u) {
-            sbyte = 255;
         }
-        uint32_t w = code << (4 * (lane & 7));
-        w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-        w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-        w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
-        if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pc + 16 * p + 4 * (lane >> 3)) = w;
-        if (lane == 0) sf[16 * p] = static_cast<uint8_t>(sbyte);
+    }
+    // Transpose the 8 x 8 nibbles of each group of 8 lanes (three butterfly
+    // exchanges): lane 8j + p then holds plane p's digits of elements
+    // 8j .. 8j+7, element 8j + i in nibble i -- one 32-bit word per lane, stored
+    // by every lane at once.
+#pragma unroll
+    for (int bs = 4; bs >= 1; bs >>= 1) {
+        const uint32_t m = bs == 4 ? 0x0000FFFFu : (bs == 2 ? 0x00FF00FFu : 0x0F0F0F0Fu);
+        const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, bs);
+        x = (lane & bs) ? (((y & ~m) >> (4 * bs)) | (x & ~m)) : ((x & m) | ((y & m) << (4 * bs)));
+    }
+    *reinterpret_cast<uint32_t*>(pc + 16 * (lane & 7) + 4 * (lane >> 3)) = x;
+    if (lane < kMxPlanes) {
+        const int s = e0 - 2 * lane;
+        sf[16 * lane] = static_cast<uint8_t>((live && s >= -127) ? s + 127 : ((!live && lane == 0 && mb != 0u) ? 255 : 0));
     }
 }
 

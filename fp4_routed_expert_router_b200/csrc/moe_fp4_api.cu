@@ -43,7 +43,7 @@ struct moe_fp4_ctx {
     uint8_t* d_mx = nullptr;           // one allocation holding the buffers below
     MxArgs mx{};                       // its buffer pointers (xp, xsf, hp, hsf, part, seq, cnt, ready, zero)
     int* d_err = nullptr;              // error word [4]
-    unsigned int* d_ticket = nullptr;  // route kernel ticket
+    unsigned int* d_ticket = nullptr;  // route kernel barriers + per-CTA expert counts (ticket_words)
     unsigned long long timeout_ns = 1000000000ull;   // bounded device waits
     std::vector<int32_t> h_table;      // host mirror of d_table
     std::vector<int64_t> slot_owner;   // slot -> layer*E+expert or -1
@@ -135,6 +135,42 @@ cudaError_t launch_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim
         cudaEventRecord(ea, s);
     }
     cudaError_t e = launch_pdl(kern, grid, block, smem, s, args...);
+    if (prof) {
+        cudaEventRecord(eb, s);
+        c->prof.push_back({name, ea, eb});
+    }
+    return e;
+}
+
+// Words of the route kernel's grid scratch: two barriers, an exit count and a
+// failure flag, then one row of expert counts per CTA (at most one CTA per SM).
+size_t ticket_words(const moe_fp4_ctx* c) {
+    return 4 + static_cast<size_t>(c->sm_count) * static_cast<size_t>(c->cfg.n_experts);
+}
+
+// The same with a cooperative launch (all CTAs co-resident; no PDL attribute,
+// so the kernel starts once its predecessor has completed).
+template <typename Kern, typename... Args>
+cudaError_t launch_coop_k(moe_fp4_ctx* c, const char* name, Kern kern, dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, Args... args) {
+    const bool prof = c->profile && c->prof.size() < 65536;
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    if (prof) {
+        ea = take_event(c);
+        eb = take_event(c);
+        cudaEventRecord(ea, s);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
     if (prof) {
         cudaEventRecord(eb, s);
         c->prof.push_back({name, ea, eb});
@@ -374,7 +410,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
         cudaMalloc(&c->d_norm, sizeof(float) * (ent > 0 ? ent : 1)) != cudaSuccess ||
         cudaMalloc(&c->d_grp, sizeof(int32_t) * (2 * static_cast<size_t>(cfg->n_experts) + 1 + ent)) != cudaSuccess ||
         cudaMalloc(&c->d_err, sizeof(int) * 4) != cudaSuccess ||
-        cudaMalloc(&c->d_ticket, sizeof(unsigned int)) != cudaSuccess) {
+        cudaMalloc(&c->d_ticket, sizeof(unsigned int) * ticket_words(c)) != cudaSuccess) {
         cudaGetLastError();
         return bail(MOE_FP4_ENOMEM);
     }
@@ -400,7 +436,7 @@ moe_fp4_status moe_fp4_create(const moe_fp4_config* cfg, int device, void* arena
     if (cudaMemset(c->d_table, 0xFF, sizeof(int32_t) * L * E) != cudaSuccess ||
         cudaMemset(c->d_rowref, 0, rowref_bytes) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(int) * 4) != cudaSuccess ||
-        cudaMemset(c->d_ticket, 0, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(c->d_ticket, 0, sizeof(unsigned int) * ticket_words(c)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
         return bail(MOE_FP4_ECUDA);
     c->h_table.assign(L * E, -1);
@@ -591,9 +627,10 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx* c, int layer, const float* logits, con
     if ((T > 0 && (!logits || !ids || !weights || !perm)) || !counts || !offsets)
         return host_fail(c, MOE_FP4_EINVAL, "route: NULL output");
     RouteArgs a{logits, keep_mask, T, g.n_experts, g.top_k, ids, weights, counts, offsets, perm,
-                c->d_ticket, c->d_err};
-    const unsigned grid = T > 0 ? static_cast<unsigned>((T + kRouteWarps - 1) / kRouteWarps) : 1u;
-    const size_t smem = sizeof(int) * kRouteWarps * g.n_experts;
+                c->d_ticket, c->d_err, c->timeout_ns};
+    int want = T > 0 ? (T + kRouteWarps - 1) / kRouteWarps : 1;   // a warp per token, up to one CTA per SM
+    const unsigned grid = static_cast<unsigned>(want < c->sm_count ? want : c->sm_count);
+    const size_t smem = sizeof(int) * (2 * static_cast<size_t>(g.n_experts) + 1);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (T * g.top_k <= 32) {   // one warp: route + bitonic grouping
@@ -604,11 +641,11 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx* c, int layer, const float* logits, con
         else
             e = launch_k(c, "route", route_small_kernel<32>, dim3(1), dim3(32), 0, s, a);
     } else if (g.n_experts <= 128)
-        e = launch_k(c, "route", route_kernel<4>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+        e = launch_coop_k(c, "route", route_grid_kernel<4>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
     else if (g.n_experts <= 384)
-        e = launch_k(c, "route", route_kernel<12>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+        e = launch_coop_k(c, "route", route_grid_kernel<12>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
     else
-        e = launch_k(c, "route", route_kernel<32>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
+        e = launch_coop_k(c, "route", route_grid_kernel<32>, dim3(grid), dim3(kRouteWarps * 32), smem, s, a);
     return e == cudaSuccess ? MOE_FP4_OK : cuda_fail(c, e, "route: launch");
 }
 
@@ -770,7 +807,7 @@ moe_fp4_status moe_fp4_saliency(moe_fp4_ctx* c, int T, const float* weights, con
                              static_cast<const float*>(c->d_o), n_ent, g.hidden, c->d_norm);
     if (e != cudaSuccess) return cuda_fail(c, e, "saliency: norm launch");
     e = launch_k(c, "saliency", saliency_kernel, dim3((g.n_experts + 127) / 128), dim3(128), 0, s,
-                 static_cast<const float*>(c->d_norm), weights, offsets, perm, g.n_experts, saliency);
+                 static_cast<const float*>(c->d_norm), weights, offsets, perm, g.n_experts, n_ent, saliency);
     if (e != cudaSuccess) return cuda_fail(c, e, "saliency: launch");
     return MOE_FP4_OK;
 }

@@ -13,11 +13,14 @@
 // histograms with warp-aggregated updates (match_any), an exclusive scan,
 // and a second, ordered pass that places each entry.
 //
-// Launch: one warp per token, 8 tokens per CTA.  The CTA that finishes last
-// (a release/acquire ticket) runs the grouping over all T*k entries, so route
-// is a single kernel whatever T is.
+// Launch: one kernel whatever T is.  Up to 32 entries, one warp routes and
+// sorts (route_small_kernel).  Beyond that a grid of co-resident CTAs
+// (cooperative launch, at most one per SM) routes contiguous token ranges and
+// groups all T*k entries together in three phases split by two bounded grid
+// barriers (route_grid_kernel); no CTA ever walks all entries alone.
 #pragma once
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -42,8 +45,10 @@ struct RouteArgs {
     int32_t* counts;
     int32_t* offsets;
     int32_t* perm;
-    unsigned int* ticket;   // zero between launches
+    unsigned int* ticket;   // [4 + grid * E]: two grid barriers, an exit count and a failure flag (zero
+                            // between launches), then the per-CTA expert counts of route_grid_kernel
     int* err;
+    unsigned long long timeout_ns;   // limit of each grid-barrier wait (route_grid_kernel)
 };
 
 // Top-k of one token's logits by one warp: writes the k chosen experts (in
@@ -184,35 +189,161 @@ __global__ void __launch_bounds__(kRouteWarps * 32) group_kernel(RouteArgs a) {
     pdl_trigger();
 }
 
-template <int NI>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
-    extern __shared__ int smem_hist[];
-    __shared__ int is_last;
-    pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kRouteWarps + warp;
-    if (t < a.T) route_token<NI>(a, t, lane);
-    if (gridDim.x == 1) {        // the only CTA: no ticket needed
-        __syncthreads();
-        group_entries(a, smem_hist);
-        pdl_trigger();
-        return;
-    }
+// Grid barrier over gridDim.x co-resident CTAs, called by all threads of the
+// CTA: every thread's earlier global writes are published before thread 0
+// arrives (release), and none of the CTA reads data of this phase before
+// thread 0 has seen all arrivals (acquire).  Bounded: gives up after
+// timeout_ns and returns false (the same answer in every thread).
+__device__ __forceinline__ bool route_grid_sync(unsigned int* bar, unsigned long long timeout_ns, int* ok_s) {
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        unsigned int prev;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.ticket) : "memory");
-        is_last = (prev == gridDim.x - 1);
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+        const uint64_t t0 = global_timer_ns();
+        int ok = 1;
+        for (;;) {
+            unsigned int v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= gridDim.x) break;
+            if (global_timer_ns() - t0 > timeout_ns) { ok = 0; break; }
+            __nanosleep(64);
+        }
+        *ok_s = ok;
     }
     __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    group_entries(a, smem_hist);
-    pdl_trigger();
-    if (threadIdx.x == 0) *a.ticket = 0;
+    return *ok_s != 0;
 }
 
+// Route and group T*k entries on a grid of G co-resident CTAs (cooperative
+// launch).  CTA c owns the tokens [c*tpc, (c+1)*tpc), so its entries are one
+// contiguous range, and the phases are:
+//   1. one warp per token routes; the CTA counts its entries per expert in
+//      shared memory and publishes the row cnt[c][0..E);
+//   2. one warp per expert: the exclusive prefix of cnt[.][e] over the CTAs in
+//      CTA order (in place) and the expert's total, counts[e];
+//   3. every CTA scans counts into offsets (CTA 0 stores them) and places its
+//      own entries in order at offsets[e] + cnt[c][e] + (earlier entries of e
+//      in the CTA).
+// This is the stable order of group_entries: by expert, then by entry index.
+// A barrier wait that gives up latches ETIMEOUT and ends the CTA's work.  The
+// last CTA to leave clears the barrier words for the next launch and, if any
+// CTA gave up, overwrites the grouping with an empty one (zero counts and
+// offsets, perm = identity), so that the kernels after it find a valid
+// routing with no work instead of whatever the outputs held before.
+// smem: int [2E + 1] (the CTA's counts, then the offsets).
+template <int NI>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_grid_kernel(RouteArgs a) {
+    extern __shared__ int smem_route[];
+    __shared__ int ok_s;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k, G = gridDim.x, c = blockIdx.x;
+    unsigned int* bar = a.ticket;                    // [0], [1] barriers, [2] exits, [3] a CTA gave up
+    int* cnt = reinterpret_cast<int*>(a.ticket + 4);  // [G][E]
+    int* hist = smem_route;                           // [E]
+    int* offs = smem_route + E;                       // [E + 1]
+    const int tpc = (a.T + G - 1) / G;
+    const int t0 = min(a.T, c * tpc), t1 = min(a.T, t0 + tpc);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    pdl_wait();
+    // phase 1
+    for (int t = t0 + warp; t < t1; t += kRouteWarps) route_token<NI>(a, t, lane);
+    __syncthreads();
+    for (int i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x) atomicAdd(&hist[a.ids[i]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[static_cast<size_t>(c) * E + e] = hist[e];
+    bool ok = route_grid_sync(bar + 0, a.timeout_ns, &ok_s);
+    // phase 2
+    if (ok) {
+        for (int e = c * kRouteWarps + warp; e < E; e += G * kRouteWarps) {
+            int run = 0;
+            for (int b = 0; b < G; b += 32) {
+                const int cc = b + lane;
+                const int v = (cc < G) ? __ldcg(cnt + static_cast<size_t>(cc) * E + e) : 0;
+                int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += u;
+                }
+                if (cc < G) cnt[static_cast<size_t>(cc) * E + e] = run + incl - v;
+                run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            }
+            if (lane == 0) a.counts[e] = run;
+        }
+        ok = route_grid_sync(bar + 1, a.timeout_ns, &ok_s);
+    }
+    // phase 3
+    if (ok) {
+        if (warp == 0) {   // exclusive scan of counts over experts, per-lane runs of consecutive experts
+            const int per = (E + 31) / 32;
+            int local = 0;
+            for (int q = 0; q < per; ++q) {
+                const int e = lane * per + q;
+                if (e < E) local += __ldcg(a.counts + e);
+            }
+            int incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            int run = incl - local;
+            for (int q = 0; q < per; ++q) {
+                const int e = lane * per + q;
+                if (e < E) {
+                    offs[e] = run;
+                    run += __ldcg(a.counts + e);
+                }
+            }
+            if (lane == 31) offs[E] = run;
+        }
+        __syncthreads();
+        if (c == 0)
+            for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = offs[e];
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            if (hist[e] > 0) hist[e] = offs[e] + __ldcg(cnt + static_cast<size_t>(c) * E + e);
+        __syncthreads();
+        if (warp == 0) {
+            for (int b = t0 * k; b < t1 * k; b += 32) {
+                const int i = b + lane;
+                const int e = (i < t1 * k) ? a.ids[i] : -1;
+                const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+                const int base = (e >= 0) ? hist[e] : 0;
+                __syncwarp();
+                if (e >= 0) {
+                    a.perm[base + __popc(peers & lanemask_lt())] = i;
+                    if (lane == __ffs(peers) - 1) hist[e] = base + __popc(peers);
+                }
+                __syncwarp();
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        latch_error(a.err, ERR_ETIMEOUT, c, KID_ROUTE);
+        atomicOr(bar + 3, 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {   // the last CTA out clears the barrier words (no CTA waits on them any more)
+        unsigned int prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(bar + 2) : "memory");
+        ok_s = 0;
+        if (prev == static_cast<unsigned int>(G) - 1) {
+            ok_s = (atomicAdd(bar + 3, 0u) != 0u) ? 2 : 1;   // 2: some CTA gave up
+            bar[0] = 0;
+            bar[1] = 0;
+            bar[2] = 0;
+            bar[3] = 0;
+        }
+    }
+    __syncthreads();
+    if (ok_s == 2) {   // every other CTA has left: replace the grouping by an empty one
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+            a.offsets[e] = 0;
+            if (e < E) a.counts[e] = 0;
+        }
+        for (int i = threadIdx.x; i < a.T * k; i += blockDim.x) a.perm[i] = i;
+    }
+    pdl_trigger();
+}
 
 // ---------------------------------------------------------------------------
 // Small batches (T*k <= 32): one warp routes the tokens, then groups the

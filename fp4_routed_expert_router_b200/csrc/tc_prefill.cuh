@@ -170,7 +170,14 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* x, con
     pdl_trigger();
     const int row = blockIdx.x;
     if (row >= n_rows) return;
-    const int src = __ldg(perm + row) / k;
+    const int ent = __ldg(perm + row);
+    if (ent < 0 || ent >= n_rows) {   // not an entry of this batch (an invalid routing): a zero row
+        uint32_t* d = reinterpret_cast<uint32_t*>(xg + static_cast<size_t>(row) * H);
+        for (int i = threadIdx.x; i < H / 2; i += blockDim.x) d[i] = 0u;
+        if (threadIdx.x == 0) colscale[row] = 0.0f;
+        return;
+    }
+    const int src = ent / k;
     const uint32_t* s = reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(src) * H);
     uint32_t mx = 0;
     for (int i = threadIdx.x; i < H / 2; i += blockDim.x) mx = max(mx, bf16x2_absmax(s[i]));
@@ -286,7 +293,11 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             for (int base = 0; base < E; base += 32) {
                 const int e = base + lane;
                 const int o0 = (e < E) ? offs_s[e] : 0, o1 = (e < E) ? offs_s[e + 1] : 0;
-                const bool on = (e < E) && (o1 > o0);
+                bool on = (e < E) && (o1 > o0);
+                if (on && (o0 < 0 || o1 > t.T * a.k)) {   // not a grouping of these T*k entries
+                    latch_error(a.err, ERR_EINVAL, e, UP ? KID_TC_UP : KID_TC_DOWN);
+                    on = false;
+                }
                 const uint32_t ball = __ballot_sync(0xFFFFFFFFu, on);
                 const int pos = n + __popc(ball & lanemask_lt());
                 const int mine = on ? n_mt * ((o1 - o0 + kTcNmax - 1) / kTcNmax) : 0;
@@ -440,6 +451,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                         const int jt = c16 * 16 + qq;
                         if (jt < nvalid) {
                             const int entn = __ldg(a.perm + p0 + n0 + jt);
+                            if (entn < 0 || entn >= t.T * a.k) continue;   // not an entry of this batch
                             const float cs = __ldg(t.colscale + p0 + n0 + jt);
                             a.obuf[static_cast<size_t>(entn) * a.H + mt * OUT_ROWS + 32 * lg + lane] =
                                 (slot >= 0) ? __uint_as_float(v[qq]) * rowmul * cs : 0.0f;

@@ -216,7 +216,12 @@ moe_fp4_status moe_fp4_residency_stats(moe_fp4_ctx *ctx, int64_t *stats);
  *  perm      int32 [T*k] out: entry indices t*k+j grouped by expert, ascending
  *            (t, j) inside each expert (a stable counting sort).
  * `layer` is accepted for symmetry with forward and must be in [0, L).
- * T = 0 writes zero counts and offsets.  Errors: EINVAL, ECUDA.
+ * T = 0 writes zero counts and offsets.  Above 32 entries (T*k) the launch is
+ * cooperative: up to one CTA per SM, which route contiguous token ranges and
+ * meet at two bounded grid barriers to group the entries (a barrier that
+ * gives up latches ETIMEOUT).  Route calls of one context share those barrier
+ * words, so they must not overlap on the GPU (one stream, or ordered streams).
+ * Errors: EINVAL, ECUDA; latched EINVAL, ETIMEOUT.
  */
 moe_fp4_status moe_fp4_route(moe_fp4_ctx *ctx, int layer, const float *logits,
                              const uint8_t *keep_mask, int T, int32_t *ids, float *weights,
@@ -231,14 +236,17 @@ moe_fp4_status moe_fp4_route(moe_fp4_ctx *ctx, int layer, const float *logits,
  *  x_out     bf16 [T, H] out or NULL, 8-byte aligned: bf16_rne(x + y), the
  *            residual update of a stacked layer; may alias x.
  * An entry routed to an expert with no slot contributes zero and latches
- * ESLOT.  Scratch (prescaled x and h rows, per-entry fp32 outputs and the
- * decode kernel's barrier counters) lives in the context's workspace, so calls
+ * ESLOT.  Offsets outside [0, T*k] latch EINVAL and that expert contributes
+ * nothing; perm entries outside [0, T*k) are skipped, so an invalid grouping
+ * gives wrong outputs and an error, never an access outside the buffers.
+ * Scratch (digit planes, prescaled x and h rows, per-entry fp32 outputs and
+ * the decode kernel's counters) lives in the context's workspace, so calls
  * on one context must not overlap in time.
- * Path: while 4*T*k < 3*E one persistent kernel runs the
- * whole layer -- w1/w3 GEMV with SwiGLU, w2 GEMV and, for T <= 16, the
- * combine -- with one CTA per SM launched cooperatively; larger batches run
- * the tcgen05 grouped GEMMs.  MOE_FP4_OPT_PATH overrides the choice.
- * Errors: EINVAL, ECUDA.
+ * Path: while 4*T*k < 3*E one persistent kernel runs the whole layer on the
+ * block-scaled FP4 tensor cores -- w1/w3 with SwiGLU, w2 and, for T <= 16,
+ * the combine -- with one CTA per SM launched cooperatively; larger batches
+ * run the tcgen05 grouped GEMMs.  MOE_FP4_OPT_PATH overrides the choice.
+ * Errors: EINVAL, ECUDA; latched EINVAL, ESLOT, ETIMEOUT.
  */
 moe_fp4_status moe_fp4_forward(moe_fp4_ctx *ctx, int layer, const uint16_t *x, int T,
                                const int32_t *ids, const float *weights,
