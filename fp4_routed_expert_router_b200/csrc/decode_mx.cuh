@@ -95,18 +95,13 @@ constexpr int kMxPlaneTile = 512;                 // one row's planes for 128 K:
 constexpr int kMxPlaneScale = 128;                // their scales: [8 planes][16 B], byte b = block b
 constexpr int kMxOffB = kUnitBytes;               // slot: A codes | A scales | B (g x 512) | B scale rows (g x 128)
 constexpr int kMxMaxSlots = 24;
-constexpr int kMxPrefetchLaps = 0;                // weights prefetched into L2 this many ring laps ahead
-                                                  // (0: none -- two laps measured slower at batch 1 on B200)
 constexpr int kMxRouteMax = 64;                   // T*k routed inside the kernel at most
 constexpr int kMxRouteExperts = 384;              // E routed inside the kernel at most
 constexpr int kMxCombineMax = 16;                 // tokens combined inside the kernel at most
 constexpr int kMxMaxEntries = 768;                // token-expert entries of one launch at most (workspace)
-constexpr int kMxChunks = 1;                      // chunks of token groups in the schedule (see the work section)
-constexpr int kMxLag = 2;                         // down(c) runs after up(c + kMxLag)
 constexpr int kMxPartUp = 2 * kMxGroup * 128;     // floats of one up side (w1 then w3)
 constexpr int kMxPartDown = kMxGroup * 128;       // floats of one down side
-constexpr int kMxPartChunk = 2 * kMxPartUp + 2 * kMxPartDown;   // per chunk: 2 up sides, 2 down sides
-constexpr int kMxPartFloats = kMxChunks * kMxPartChunk;         // split-item partials of one CTA
+constexpr int kMxPartFloats = 2 * kMxPartUp + 2 * kMxPartDown;  // split-item partials of one CTA: 2 up, 2 down sides
 constexpr uint32_t kMxTmemCols = 512;             // accumulators [2][issuer][16 g] columns, scale atoms at 384 + 8 w
 
 struct MxArgs {
@@ -538,18 +533,16 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
     mx_fence_after();
 
     // ------------------------------------------------------------ work
-    // The groups form C = min(n_gs, kMxChunks) chunks; each chunk's up units,
-    // and its down units, are split contiguously over all CTAs, and every CTA
-    // runs its segments in the order up(0) .. up(L-1), then up(c), down(c - L)
-    // for c = L .. C-1, then the last L downs.  With kMxChunks = 1 (the setting
-    // used) that is all up units, then all down units: a staggered order with
-    // six chunks measured 3.4x slower at batch 1 on B200, because accumulators
-    // and the epilogue run strictly in order, so a down part waiting for
-    // another CTA's h holds up every part queued behind it.
+    // Two segments: every up unit of the batch, split contiguously over all
+    // CTAs, then every down item, dealt whole.  (Interleaving the two -- the
+    // down part of some groups after the up part of later ones -- measured
+    // 3.4x slower at batch 1 on B200: accumulators and the epilogue run in
+    // order, so a down part waiting for another CTA's h holds up every part
+    // queued behind it.)
     const int n_gs = n_gs_s;
     const unsigned int tag = tag_s;
     const int upi = 2 * KU, dpi = KD;                       // units per up / down item
-    const int C = min(n_gs, kMxChunks), n_seg = 2 * C;
+    const int n_seg = 2;
     unsigned int* x_cnt = a.cnt + static_cast<size_t>(tag & 1u) * a.cnt_cap;   // this launch's bank
     unsigned int* up_cnt = x_cnt + 1;
     unsigned int* dn_cnt = up_cnt + p.max_up_items;
@@ -559,29 +552,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
         const int ent = routed ? r_perm[pos] : __ldg(a.perm + pos);
         return (ent >= 0 && ent < n_ent) ? ent : -1;
     };
-    // segment s: up or down, its chunk, the chunk's unit space [base, base + n)
-    // and this CTA's range [ua, ub) in it (global unit indices)
+    // segment sg (0: up, 1: down): its unit space [base, base + n) and this
+    // CTA's range [ua, ub) in it (global unit indices)
     auto segment = [&](int sg, bool& up, int& c, int& base, int& n, int& ua, int& ub) {
-        if (C <= kMxLag) {
-            up = sg < C;
-            c = up ? sg : sg - C;
-        } else if (sg < kMxLag) {
-            up = true;
-            c = sg;
-        } else {
-            const int t = sg - kMxLag;
-            if (t < 2 * (C - kMxLag)) {
-                up = (t & 1) == 0;
-                c = up ? kMxLag + (t >> 1) : (t >> 1);
-            } else {
-                up = false;
-                c = C - kMxLag + (t - 2 * (C - kMxLag));
-            }
-        }
-        const int g0 = n_gs * c / C, g1 = n_gs * (c + 1) / C;
-        const int per_group = up ? RT * upi : NT * dpi;
-        base = g0 * per_group;
-        n = (g1 - g0) * per_group;
+        up = sg == 0;
+        c = 0;
+        base = 0;
+        n = n_gs * (up ? RT * upi : NT * dpi);
         if (up) {   // up units split evenly: an item may be cut between CTAs
             ua = base + mx_range_start(n, G, b);
             ub = base + mx_range_start(n, G, b + 1);
@@ -610,8 +587,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
             const int kMxProducers = S;
             const uint64_t pol = policy_evict_first();
             // the CTA's units as segments: local index i -> global unit gu
-            int seg_first[2 * kMxChunks + 1], seg_ua[2 * kMxChunks];
-            bool seg_up[2 * kMxChunks];
+            int seg_first[3], seg_ua[2];
+            bool seg_up[2];
             int n_units = 0;
             for (int sg = 0; sg < n_seg; ++sg) {
                 int c, base, n, ua, ub;
@@ -655,20 +632,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
                         bulk_g2s(ring + static_cast<size_t>(s) * SB, a.arena + static_cast<size_t>(slot) * a.slot_bytes + uoff,
                                  kUnitBytes, &full[s], pol);
                         reinterpret_cast<volatile int*>(last_issue)[s] = i;
-                    }
-                    // optional L2 prefetch of this slot's unit kMxPrefetchLaps laps ahead (and, on the
-                    // first lap, of every lap up to that)
-                    for (int d = (mA == 0 ? 1 : kMxPrefetchLaps); kMxPrefetchLaps > 0 && d <= kMxPrefetchLaps; ++d) {
-                        const int jd = i + d * S;
-                        if (jd >= n_units) break;
-                        bool upd;
-                        int gsd, tiled, matd, kud;
-                        unit(jd, upd, gsd, tiled, matd, kud);
-                        const int sld = act_slot[gs_a[gsd]];
-                        if (sld >= 0)
-                            bulk_prefetch_l2(a.arena + static_cast<size_t>(sld) * a.slot_bytes +
-                                                 (upd ? up_unit_offset(L, matd, tiled, kud) : down_unit_offset(L, tiled, kud)),
-                                             kUnitBytes);
                     }
                     ++mA;
                     progress = true;
@@ -901,7 +864,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
                 for (int bb = bf; up && bb <= bl; ++bb) nparts += mx_range_start(n, G, bb) < mx_range_start(n, G, bb + 1);
                 if (nparts > 1) {   // split item: store this part, the last part to arrive adds them all
                     const int side = (item == first_item) ? 0 : 1;
-                    float* pp = a.part + static_cast<size_t>(b) * kMxPartFloats + c * kMxPartChunk +
+                    float* pp = a.part + static_cast<size_t>(b) * kMxPartFloats +
                                 (up ? side * kMxPartUp : 2 * kMxPartUp + side * kMxPartDown);
 #pragma unroll
                     for (int e = 0; e < kMxGroup; ++e) {
@@ -927,7 +890,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) moe_fp4_decode_mx(MxArgs a, Slo
                         const int st = mx_range_start(n, G, bb);
                         if (st == mx_range_start(n, G, bb + 1)) continue;
                         const int sd = (item == (base + st) / per) ? 0 : 1;
-                        const float* q = a.part + static_cast<size_t>(bb) * kMxPartFloats + c * kMxPartChunk +
+                        const float* q = a.part + static_cast<size_t>(bb) * kMxPartFloats +
                                          (up ? sd * kMxPartUp : 2 * kMxPartUp + sd * kMxPartDown);
 #pragma unroll
                         for (int e = 0; e < kMxGroup; ++e) {
