@@ -348,16 +348,20 @@ cudaError_t tc_forward(moe_fp4_ctx* c, const ExpertArgs& a, const SlotLayout& L,
     cudaError_t e = launch_k(c, "gather", gather_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, s,
                              a.x, a.perm, a.k, a.H, rows, p.xg, p.xcs);
     if (e != cudaSuccess) return e;
-    TcArgs tu = tc_args(p, a, L, T, true, c->d_rowref), td = tc_args(p, a, L, T, false, c->d_rowref);
+    const int nmax = tc_nmax_for(T);
+    TcArgs tu = tc_args(p, a, L, T, true, c->d_rowref, nmax), td = tc_args(p, a, L, T, false, c->d_rowref, nmax);
     if (!tu.centries || !td.centries) return cudaErrorNotSupported;
     tu.timeout_ns = td.timeout_ns = c->timeout_ns;
     const dim3 grid(static_cast<unsigned>(p.sm_count)), block(kTcThreads);
-    e = launch_k(c, "tc_up", tc_gemm_kernel<true>, grid, block, tc_smem_bytes(tu), s, tu, p.map_x);
+    const bool narrow = nmax == kTcNmaxNarrow;
+    e = launch_k(c, "tc_up", narrow ? tc_gemm_kernel<true, kTcNmaxNarrow> : tc_gemm_kernel<true, kTcNmaxWide>, grid,
+                 block, tc_smem_bytes(tu), s, tu, p.map_x);
     if (e != cudaSuccess) return e;
     e = launch_k(c, "h_convert", h_convert_kernel, dim3(static_cast<unsigned>((rows * 32 + 255) / 256)), dim3(256), 0,
                  s, static_cast<const uint16_t*>(p.hb), a.I, rows, p.hh, p.hcs);
     if (e != cudaSuccess) return e;
-    return launch_k(c, "tc_down", tc_gemm_kernel<false>, grid, block, tc_smem_bytes(td), s, td, p.map_h);
+    return launch_k(c, "tc_down", narrow ? tc_gemm_kernel<false, kTcNmaxNarrow> : tc_gemm_kernel<false, kTcNmaxWide>,
+                    grid, block, tc_smem_bytes(td), s, td, p.map_h);
 }
 
 }  // namespace

@@ -6,8 +6,9 @@
 //   up    a1 = W1 X^T, a3 = W3 X^T, h = bf16(silu(a1) * a3)   (K = H)
 //   down  o  = W2 H^T                                         (K = I)
 // Weights are the M side of tcgen05.mma (M = 128 TMEM lanes) and tokens the
-// N side (N <= 128, rounded up to 16).  A work item is (expert, row group,
-// chunk of <= 128 of the expert's tokens):
+// N side (N <= NMAX, rounded up to 16; NMAX = 128, or 64 with a deeper ring
+// for batches of at most 64 tokens).  A work item is (expert, row group,
+// chunk of <= NMAX of the expert's tokens):
 //   up    64 output rows: TMEM lane 32g + l holds w1 row 16g + l (l < 16) or
 //         w3 row 16g + l - 16 (l >= 16) -- exactly the two 16-row halves of
 //         slot block g -- so silu(a1) * a3 pairs lanes l and l + 16 of one
@@ -66,13 +67,24 @@ namespace moe {
 constexpr int kTcM = 128;          // TMEM lanes = A rows per MMA
 constexpr int kTcBK = 64;          // K of one 128-byte swizzle atom of bf16 (four K=16 MMAs)
 constexpr int kTcSK = 128;         // K per pipeline stage (two atoms, eight MMAs)
-constexpr int kTcNmax = 128;       // tokens per item (accumulator columns)
 constexpr int kTcDequantWarps = 16;
 constexpr int kTcEpiWarps = 4;
 constexpr int kTcThreads = (kTcDequantWarps + kTcEpiWarps + 3) * 32;   // + B producer, code producer, MMA
-constexpr int kTcStages = 4;       // A (TMEM, 64 columns each) / B (shared, 32 KB each) stages
-constexpr int kTcAccCols = 2 * kTcNmax;   // two accumulators of kTcNmax fp32 columns, then the A stages
 constexpr int kTcMaxEntries = 8;   // code ring entries at most
+// Tile shapes.  NMAX = tokens per item (columns of each of the two fp32
+// accumulators); the rest of the 512 TMEM columns holds the A stages (64
+// columns each), and the B ring in shared memory has as many stages
+// (2 atoms x NMAX rows x 128 bytes each):
+//   NMAX 128: 4 stages -- an expert's tokens are read in chunks of 128;
+//   NMAX  64: 6 stages -- chosen when no expert can hold more than 64 tokens
+//             (batch <= 64: a token names an expert at most once), where the
+//             deeper ring is faster (decode batch 64: 1.13 ms against 1.22 ms
+//             on B200) and no weight is read twice.  At 2048 tokens the extra
+//             chunks of hot experts cost as much as the stages gain.
+constexpr int kTcNmaxWide = 128;
+constexpr int kTcNmaxNarrow = 64;
+__host__ __device__ constexpr int tc_stages(int nmax) { return (512 - 2 * nmax) / 64; }
+static_assert(tc_stages(kTcNmaxWide) == 4 && tc_stages(kTcNmaxNarrow) == 6, "TMEM: 2 NMAX + 64 S = 512 columns");
 
 struct TcArgs {
     ExpertArgs g;
@@ -81,7 +93,8 @@ struct TcArgs {
     uint16_t* hb;           // [T*k, I] bf16 h (up output, grouped order)
     SlotLayout L;
     int T;
-    int off_b;             // dynamic smem offset of the B ring (1024-aligned), kTcStages x 2 atoms x kTcNmax rows x 128 bytes
+    int nmax;              // tile shape: kTcNmaxWide or kTcNmaxNarrow (tokens per item)
+    int off_b;             // dynamic smem offset of the B ring (1024-aligned), stages x 2 atoms x nmax rows x 128 bytes
     int off_code;          // offset of the code ring: centries x entry_bytes
     int entry_bytes;       // one code ring entry: spe units' worth of the item's rows
     int spe;               // 128-K units (= stages) per code entry: 2 when K / 128 is even, else 1
@@ -213,14 +226,15 @@ __global__ void __launch_bounds__(256) h_convert_kernel(const uint16_t* hb, int 
 }
 
 // ------------------------------------------------------------------ GEMM
-template <bool UP>
+template <bool UP, int NMAX>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     constexpr int ROWT = UP ? 4 : 8;             // 16-row groups per item
     constexpr int OUT_ROWS = UP ? 64 : 128;      // output rows per item
     constexpr int ACOLS = kTcSK / 2;             // TMEM columns of one stage's A (bf16 pairs)
-    constexpr int BATOM = kTcNmax * 128;         // bytes of one B swizzle atom (N rows x 64 K)
-    constexpr int S = kTcStages;
+    constexpr int BATOM = NMAX * 128;            // bytes of one B swizzle atom (N rows x 64 K)
+    constexpr int S = tc_stages(NMAX);
+    constexpr int ACC_COLS = 2 * NMAX;           // two accumulators of NMAX fp32 columns, then the A stages
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     // the 128-byte swizzle of the B tiles is defined on 1024-byte atoms of the
     // shared address space: align the working base explicitly
@@ -300,7 +314,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                 }
                 const uint32_t ball = __ballot_sync(0xFFFFFFFFu, on);
                 const int pos = n + __popc(ball & lanemask_lt());
-                const int mine = on ? n_mt * ((o1 - o0 + kTcNmax - 1) / kTcNmax) : 0;
+                const int mine = on ? n_mt * ((o1 - o0 + NMAX - 1) / NMAX) : 0;
                 int incl = mine;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -330,7 +344,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
     }
     pdl_trigger();
     const uint32_t tmem = tmem_base_s;
-    const uint32_t tmem_a = tmem + kTcAccCols;   // A stage st at + st * ACOLS
+    const uint32_t tmem_a = tmem + ACC_COLS;   // A stage st at + st * ACOLS
     const int n_act = n_act_s, n_work = n_work_s, G = gridDim.x;
     const int my_items = (static_cast<int>(blockIdx.x) < n_work) ? (n_work - 1 - blockIdx.x) / G + 1 : 0;
     auto item_of = [&](int i, int& ai, int& mt, int& n0) {
@@ -341,10 +355,10 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             if (wprefix[mid] <= w) lo = mid; else hi = mid - 1;
         }
         const int v = w - wprefix[lo];
-        const int chunks = (act_m[lo] + kTcNmax - 1) / kTcNmax;
+        const int chunks = (act_m[lo] + NMAX - 1) / NMAX;
         ai = lo;
         mt = v / chunks;
-        n0 = (v - mt * chunks) * kTcNmax;
+        n0 = (v - mt * chunks) * NMAX;
     };
     auto code_entry = [&](int ce) { return smem + t.off_code + static_cast<size_t>(ce) * t.entry_bytes; };
     auto stage_b = [&](int st) { return smem + t.off_b + static_cast<size_t>(st) * (2 * BATOM); };
@@ -415,7 +429,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
             const int p0 = act_p0[ai], m = act_m[ai], slot = act_slot[ai];
-            const int nvalid = min(kTcNmax, m - n0);
+            const int nvalid = min(NMAX, m - n0);
             const int ab = i & 1;
             if (!mbar_wait(&acc_full[ab], (i >> 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
                 latch_error(a.err, ERR_ETIMEOUT, i, kid);
@@ -429,7 +443,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
                                                                          emat * a.I + erow)) - 127);
             for (int c16 = 0; c16 * 16 < nvalid; ++c16) {
                 uint32_t v[16];
-                tmem_ld16(tmem + lane_addr + ab * kTcNmax + c16 * 16, v);
+                tmem_ld16(tmem + lane_addr + ab * NMAX + c16 * 16, v);
                 if (UP) {
                     // lanes 0-15: a1 of rows 16 lg + lane; lanes 16-31 hold the matching a3
 #pragma unroll
@@ -473,7 +487,7 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
         for (int i = 0; i < my_items && !stop; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
-            const int nvalid = min(kTcNmax, act_m[ai] - n0);
+            const int nvalid = min(NMAX, act_m[ai] - n0);
             const int nb = (nvalid + 15) / 16;
             const int row0 = act_p0[ai] + n0;
             for (int s = 0; s < n_stg; ++s, ++gstg) {
@@ -565,14 +579,14 @@ tc_gemm_kernel(TcArgs t, const __grid_constant__ CUtensorMap bmap) {
         for (int i = 0; i < my_items; ++i) {
             int ai, mt, n0;
             item_of(i, ai, mt, n0);
-            const int nvalid = min(kTcNmax, act_m[ai] - n0);
+            const int nvalid = min(NMAX, act_m[ai] - n0);
             const int n = (nvalid + 15) / 16 * 16;
             const uint32_t idesc = umma_idesc_f16(kTcM, n);
             const int ab = i & 1;
             if (i >= 2 && !mbar_wait(&acc_empty[ab], ((i >> 1) - 1) & 1, abort_flag, t.timeout_ns) && lane == 0)
                 latch_error(a.err, ERR_ETIMEOUT, i, kid);
             tc_fence_after();
-            const uint32_t dacc = tmem + ab * kTcNmax;
+            const uint32_t dacc = tmem + ab * NMAX;
             for (int s = 0; s < n_stg; ++s, ++gstg) {
                 const int st = gstg % S;
                 if (!mbar_wait(&full[st], (gstg / S) & 1, abort_flag, t.timeout_ns) && lane == 0)
@@ -659,8 +673,10 @@ inline cudaError_t tc_plan_create(TcPlan* p, const moe_fp4_config& cfg, uint16_t
     auto set = [&](const void* f) {
         return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_limit);
     };
-    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<true>))) != cudaSuccess) return e;
-    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<false>))) != cudaSuccess) return e;
+    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<true, kTcNmaxWide>))) != cudaSuccess) return e;
+    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<false, kTcNmaxWide>))) != cudaSuccess) return e;
+    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<true, kTcNmaxNarrow>))) != cudaSuccess) return e;
+    if ((e = set(reinterpret_cast<const void*>(tc_gemm_kernel<false, kTcNmaxNarrow>))) != cudaSuccess) return e;
     p->ready = 1;
     return cudaSuccess;
 }
@@ -683,9 +699,13 @@ inline bool tc_prefers(int T, const moe_fp4_config& cfg) {
     return 4LL * T * cfg.top_k >= 3LL * cfg.n_experts;
 }
 
+// Tile shape for a batch of T tokens: an expert holds at most T of them.
+inline int tc_nmax_for(int T) { return T <= kTcNmaxNarrow ? kTcNmaxNarrow : kTcNmaxWide; }
+
 inline TcArgs tc_args(const TcPlan& p, const ExpertArgs& g, const SlotLayout& L, int T, bool up,
-                      const uint8_t* rowref) {
+                      const uint8_t* rowref, int nmax) {
     TcArgs t{};
+    t.nmax = nmax;
     t.g = g;
     t.rowref = rowref;
     t.colscale = up ? p.xcs : p.hcs;
@@ -696,7 +716,7 @@ inline TcArgs tc_args(const TcPlan& p, const ExpertArgs& g, const SlotLayout& L,
     t.max_active = ent < g.E ? ent : g.E;
     const int head = 1024 + 256 * 16 + 4 * (5 * t.max_active + 1 + 2 * g.E + 1);
     t.off_b = (head + 1023) / 1024 * 1024;
-    t.off_code = t.off_b + kTcStages * 2 * kTcNmax * 128;
+    t.off_code = t.off_b + tc_stages(nmax) * 2 * nmax * 128;
     const int K = up ? g.H : g.I, rows = up ? g.I : g.H;
     t.spe = (K / kTcSK) % 2 == 0 ? 2 : 1;
     t.entry_bytes = t.spe * (up ? 2 * (4096 + kUnitScaleBytes) : kUnitBytes);
