@@ -20,8 +20,8 @@
 // 2^E0 < max|v| <= 2^(E0+1), plane p holds digits d in {0, +-0.5 .. +-2} at
 // scale 2^(E0 - 2p) (a UE8M0 block scale), chosen greedily by rounding the
 // remainder to the nearest half; each remainder is at most a quarter of the
-// plane's unit, so after 8 planes it is below 2^(E0-16) < max|v| * 2^-16,
-// and every element within 2^9 of the block maximum is represented exactly
+// plane's unit, so after 8 planes it is at most 2^(E0-16) < max|v| * 2^-16,
+// and every element within 2^8 of the block maximum is represented exactly
 // (bf16 has 8 significant bits).  The planes are the N columns of the MMA
 // (8 per entry); the epilogue adds them in fp32.  Power-of-two rescalings of
 // a row rescale its planes exactly (the digits depend on v / 2^E0 only).
