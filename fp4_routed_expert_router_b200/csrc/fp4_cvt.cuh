@@ -9,7 +9,7 @@
 // instruction (cvt.rn.f16x2.e2m1x2; low nibble -> low half).  Every E2M1
 // value (0, +-0.5 .. +-6) is an f16 number, so the conversion is exact; the
 // f16 path then multiplies a block by 2^(s - s_ref) of its row (exact while
-// the row's scales span at most 24 binades) and the fp32 result by
+// the row's scales span at most 23 binades) and the fp32 result by
 // 2^(s_ref - 127).
 //
 // Activations.  The tensor-core operands are f16, the activations bf16.  A

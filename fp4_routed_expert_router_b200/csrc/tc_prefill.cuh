@@ -23,7 +23,7 @@
 //                slot_layout.cuh) and the block's scale byte, converts the
 //                codes to f16 (exact E2M1), multiplies them by 2^(s - s_ref) with
 //                s_ref the row's largest scale (exact while the row's scales
-//                span at most 24 binades: f16 reaches 2^-24), and writes them
+//                span at most 23: 0.5 * 2^-23 is f16's 2^-24), and writes them
 //                to the stage's A columns in TMEM with tcgen05.st (lane =
 //                row, two f16 per column, K in natural order).
 //   warps 16-19  epilogue: tcgen05.ld of the finished accumulator (double
