@@ -56,7 +56,8 @@ def parse():
     return p.parse_args()
 
 
-def workload_config(wl: synth.Workload, graph: bool) -> dict:
+def workload_config(wl: synth.Workload) -> dict:
+    """The workload a line measures; identical for both arms (how it is launched is reported apart)."""
     return {
         "workload": f"{wl.name}: one DeepSeek-V4.1-Flash routed-expert layer, {wl.notes}",
         "hidden": wl.hidden, "inter": wl.inter, "n_experts": wl.n_experts, "top_k": wl.top_k,
@@ -67,11 +68,14 @@ def workload_config(wl: synth.Workload, graph: bool) -> dict:
         "l2": "flushed between timed steps (2x L2 write, then its lines discarded); the step's small inputs "
               "(x, logits) are written after the flush, as the preceding layer leaves them, the expert "
               "weights come from HBM",
-        "launch": ("cuda graph of moe_fp4_route_forward" if graph else "eager moe_fp4_route_forward") +
-                  (" (one persistent kernel per step)" if wl.tokens * wl.top_k <= 64 else
-                   " (route kernel, then the expert kernels)"),
         "parallelism": "replicas (one independent layer per GPU)",
     }
+
+
+def launch_desc(wl: synth.Workload, graph: bool) -> str:
+    return (("cuda graph of moe_fp4_route_forward" if graph else "eager moe_fp4_route_forward") +
+            (" (one persistent kernel per step)" if wl.tokens * wl.top_k <= 64 else
+             " (route kernel, then the expert kernels)"))
 
 
 # ============================================================================ oracle arm
@@ -132,7 +136,8 @@ def run_reference(args, wl):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(wl, False),
+            "data": "synthetic", "config": workload_config(wl),
+            "launch": "fp64 oracle on the host cores (OpenMP over token-expert pairs)",
             "cpu_baseline": {"value": value, "unit": "tok/s", "cores": n_threads, "kind": "oracle",
                              "sample": f"{args.steps} steps x {swl.tokens} token(s) of {wl.name}"},
             "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -660,7 +665,7 @@ def run_ours(args, wl):
         "metric": METRIC, "value": toks / (total_ms * 1e-3), "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(wl, not args.no_graph),
+        "data": "synthetic", "config": workload_config(wl), "launch": launch_desc(wl, not args.no_graph),
         "hbm_gbs_step": s["hbm_gbs_step"], "hbm_frac_step": s["hbm_frac_step"],
         "kernel_ms": s["kernel_ms"],
         "roofline": s["roofline"],
