@@ -1,6 +1,7 @@
 """Expert-parallel execution of one routed-expert layer over a process group.
 
-Rank r of G holds experts [r*E/G, (r+1)*E/G) in its arena.  Each rank routes
+Rank r of G holds experts [r*S, min((r+1)*S, E)) in its arena, S = ceil(E/G)
+(so the last ranks may hold fewer, or none, when G does not divide E).  Each rank routes
 its own tokens; the (token, selected expert) entries then take one exchange
 step to the ranks owning their experts and the expert outputs take one
 exchange step back, after which each rank combines its tokens' outputs:
@@ -50,7 +51,7 @@ class DispatchPlan:
 
 
 class ExpertParallel:
-    """Contiguous expert shards: rank r owns experts [r*E/G, (r+1)*E/G)."""
+    """Contiguous expert shards: rank r owns experts [r*S, min((r+1)*S, E)), S = ceil(E/G)."""
 
     def __init__(self, n_experts: int, top_k: int, hidden: int, group=None, max_tokens: int | None = None):
         """max_tokens: the most tokens any rank brings to one layer; it sets the
@@ -60,13 +61,14 @@ class ExpertParallel:
         self.max_tokens = max_tokens
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
-        if n_experts % self.world:
-            raise ValueError(f"{n_experts} experts do not split evenly over {self.world} ranks")
+        if n_experts < 1:
+            raise ValueError("no experts to shard")
         self.E, self.k, self.H = n_experts, top_k, hidden
-        self.per_rank = n_experts // self.world
+        self.per_rank = -(-n_experts // self.world)        # ceil: expert e lives on rank e // per_rank
 
     def owned(self) -> range:
-        return range(self.rank * self.per_rank, (self.rank + 1) * self.per_rank)
+        lo = min(self.rank * self.per_rank, self.E)
+        return range(lo, min(lo + self.per_rank, self.E))
 
     def plan(self, ids: torch.Tensor, device) -> DispatchPlan:
         """Send order and counts for this rank's routed ids [T, k]; the counts
@@ -118,7 +120,10 @@ class ExpertParallel:
         width = rows.element_size()
         for d in shape:
             width *= d
-        flat = rows.contiguous().reshape(rows.shape[0], width // rows.element_size()).view(torch.uint8)
+        if rows.shape[0] == 0:   # nothing to send (an empty tensor's strides need not allow the byte view)
+            flat = torch.empty((0, width), dtype=torch.uint8, device=rows.device)
+        else:
+            flat = rows.contiguous().reshape(rows.shape[0], width // rows.element_size()).view(torch.uint8)
         out = torch.empty((sum(recv), width), dtype=torch.uint8, device=rows.device)
         dist.all_to_all_single(out, flat, recv, send, group=self.group)
         return out.view(rows.dtype).reshape((sum(recv),) + shape)
@@ -128,7 +133,8 @@ class ExpertParallel:
         """x [T, H] (bf16 bits), ids/weights [T, k] of this rank's tokens.
         expert_fn(x_rows [n, H], experts [n] int32) -> o [n, H] fp32 for
         experts this rank owns, rows with expert id -1 being empty slots (their
-        o rows are never read); combine_fn(o [T*k, H], weights) -> y [T, H].
+        o rows are never read), and n may be 0 (a rank that received nothing);
+        combine_fn(o [T*k, H], weights) -> y [T, H].
         device_plan: True / False forces a plan; None takes the device plan
         when its exchange buffer is at most DEVICE_PLAN_MAX_BYTES.  Every rank
         must take the same plan; the default depends only on the constructor's
@@ -149,10 +155,7 @@ class ExpertParallel:
         e_send = ids.reshape(-1).to(torch.int32).index_select(0, order_dev.to(ids.device)).to(x.device)
         x_recv = self._exchange(x_send, p.send_counts, p.recv_counts)
         e_recv = self._exchange(e_send, p.send_counts, p.recv_counts)
-        if x_recv.shape[0]:
-            o_recv = expert_fn(x_recv, e_recv)
-        else:
-            o_recv = torch.empty((0, self.H), dtype=torch.float32, device=x.device)
+        o_recv = expert_fn(x_recv, e_recv)      # zero rows too: every rank's o rows get expert_fn's dtype
         o_back = self._exchange(o_recv, p.recv_counts, p.send_counts)
         o = torch.empty((T * self.k, self.H), dtype=o_back.dtype, device=o_back.device)
         o[order_dev.to(o.device)] = o_back

@@ -87,7 +87,9 @@ def _rank_main(rank, world, port, tokens_per_rank, device_plan, out):
 
 
 @pytest.mark.parametrize("device_plan", [False, True])
-@pytest.mark.parametrize("world,tokens", [(2, [5, 3]), (4, [4, 0, 7, 2])])
+@pytest.mark.parametrize("world,tokens", [(2, [5, 3]), (4, [4, 0, 7, 2]),
+                                          (3, [5, 2, 4]),         # 8 experts as 3 + 3 + 2
+                                          (5, [3, 1, 0, 4, 2])])  # 2 + 2 + 2 + 2 + 0: a rank owns none
 def test_expert_parallel_matches_single_process(world, tokens, device_plan):
     import oracle
     ctx = mp.get_context("spawn")
