@@ -696,8 +696,7 @@ inline void tc_plan_destroy(TcPlan* p) {
 
 // The tcgen05 path pays off once the batch holds about as many token-expert
 // pairs as there are experts (measured crossover on B200: between 8 and 64
-// tokens at k = 6, E = 384; 64 tokens run 1.15 ms here against 1.32 ms on
-// the GEMV path).
+// tokens at k = 6, E = 384).
 inline bool tc_prefers(int T, const moe_fp4_config& cfg) {
     return 4LL * T * cfg.top_k >= 3LL * cfg.n_experts;
 }

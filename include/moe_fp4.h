@@ -71,7 +71,7 @@ typedef struct {
 /* Execution-path override for moe_fp4_set_option(MOE_FP4_OPT_PATH, .). */
 enum {
     MOE_FP4_PATH_AUTO = 0,  /* decode kernel while 4*T*k < 3*E, tcgen05 GEMM from there on */
-    MOE_FP4_PATH_GEMV = 1,  /* always the decode kernel (grouped mma.sync GEMV) */
+    MOE_FP4_PATH_GEMV = 1,  /* always the decode kernel (one persistent block-scaled FP4 tcgen05 kernel; T*k <= 768) */
     MOE_FP4_PATH_TC = 2     /* always the tcgen05 grouped GEMM */
 };
 /* Options for moe_fp4_set_option. */
@@ -145,7 +145,7 @@ moe_fp4_status moe_fp4_set_option(moe_fp4_ctx *ctx, int option, int value);
 /*
  * Per-kernel device times of the profiled launches since the last read:
  * synchronises the device, writes up to `max` records (names[i] points at a
- * static string such as "gemv_up", ms[i] its event-measured duration in
+ * static string such as "decode_layer" or "tc_up", ms[i] its event-measured duration in
  * milliseconds) and returns the number of records (0 when profiling is off),
  * or -1 on a CUDA error.  Reading clears the record list.
  */

@@ -45,8 +45,9 @@ def test_tiny_layer_parity(tiny, T):
 @pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_TC])
 @pytest.mark.parametrize("T", [1, 5, 33, 130])
 def test_tiny_forced_paths(tiny, path, T):
-    """Both expert-FFN engines on the same inputs: the register-decoded GEMV and
-    the tcgen05 grouped GEMM (token chunks of 1..128, ragged tails)."""
+    """Both expert-FFN engines on the same inputs: the decode kernel (block-scaled
+    FP4 tensor cores) and the tcgen05 f16 grouped GEMM (token chunks of 1..128,
+    ragged tails)."""
     wl = tiny.wl
     logits, mask, x, r, y = _run(tiny, T, step=1000 + T, path=path)
     ids, w = check_routing(r, logits, wl.top_k, wl.n_experts, mask)

@@ -2,7 +2,7 @@
 drafter model's expert count and fan-out as ai-shiz.ru "DeepSeek-V4.1-Flash
 дома" describes it, section "Что за модель"), at the layer's hidden 5120 /
 inter 2304.  The same kernels serve it: the 128-expert router instantiation,
-the GEMV path for small batches and the tcgen05 path for large ones."""
+the decode kernel for small batches and the tcgen05 path for large ones."""
 import numpy as np
 import pytest
 
