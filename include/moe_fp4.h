@@ -93,22 +93,22 @@ enum {
  *
  * The checkpoint stores an expert as codes first, scales after (w1, w3, w2
  * codes, then s1, s3, s2; the article's section "SSD读取性能"); the loaders
- * take that layout.  Inside a slot the same bytes are rearranged so that the
- * kernels stream one contiguous, 16-byte-aligned range per unit of work:
- *  up blocks, for each 16-row tile rt of W1/W3 and each K block f of KBu
- *  (256 when it divides H, else 128) columns, in order (rt, f):
- *      [w1 16 rows x KBu/2][w3 16 rows x KBu/2][s1 16 x KBu/32][s3 16 x KBu/32]
- *  then down blocks, for each 16-row tile of W2 and each K block of KBd
- *  (256 when it divides I, else 128):  [w2 16 rows x KBd/2][s2 16 x KBd/32]
- * so one 16-row x KBu block of w1+w3 (4,352 bytes for V4.1) and 16 rows of
- * w2 over all of I (19,584 bytes) are each contiguous.  Code bytes keep the
- * checkpoint's nibbles, but inside each 64-byte group of a row (128 K = four
- * 32-K scale blocks) the sixteen 32-bit words are transposed: 16-byte chunk c
- * holds, as its word j, codes K = 32j + 8c .. +7 of the group, which hands one
- * MMA lane column eight codes of each scale block.  In code rows of 128-byte
- * multiples the 16-byte chunk q of row r sits at q ^ ((r & 7) ^ ((r & 1) << 2))
- * (bank-conflict-free loads).  Scale bytes are stored as they are.  The total
- * is unchanged.
+ * take that layout.  Inside a slot the same bytes are regrouped into units,
+ * each one 128-row x 128-K tile of one matrix, codes and scales together,
+ * 8,704 contiguous bytes (16-byte aligned) that one bulk copy moves:
+ *  up units    for mat in (w1, w3), row tile rt < I/128, K unit ku < H/128,
+ *              at ((mat * I/128 + rt) * H/128 + ku) * 8704;
+ *  down units  after them, for row tile nt < H/128, K unit ku < I/128,
+ *              at up_bytes + (nt * I/128 + ku) * 8704, up_bytes =
+ *              2 * (I/128) * (H/128) * 8704;
+ *  in a unit   code of row r, K k (0..127): byte (r/8)*512 + (k/32)*128 +
+ *              (r%8)*16 + (k%32)/2, nibble k & 1 (low = even K, as in the
+ *              checkpoint) -- the tensor cores' K-major, no-swizzle operand
+ *              layout for 4-bit types; scale of row r, 32-K block b:
+ *              byte 8192 + (r%32)*16 + (r/32)*4 + b -- the tile one
+ *              tcgen05.cp .32x128b.warpx4 puts in tensor memory.
+ * H and I must be multiples of 128.  The total is unchanged (V4.1: 2,160
+ * units).
  */
 size_t moe_fp4_slot_bytes(const moe_fp4_config *cfg);
 
