@@ -10,9 +10,9 @@
 // for batches of at most 64 tokens).  A work item is (expert, row group,
 // chunk of <= NMAX of the expert's tokens):
 //   up    64 output rows: TMEM lane 32g + l holds w1 row 16g + l (l < 16) or
-//         w3 row 16g + l - 16 (l >= 16) -- exactly the two 16-row halves of
-//         slot block g -- so silu(a1) * a3 pairs lanes l and l + 16 of one
-//         warp (a shuffle, no shared memory);
+//         w3 row 16g + l - 16 (l >= 16) of the item's 64 rows (half of a
+//         128-row unit of each) -- so silu(a1) * a3 pairs lanes l and l + 16
+//         of one warp (a shuffle, no shared memory);
 //   down  128 output rows, lane r = row r.
 // Both GEMMs therefore run the same pipeline on a 128 x 128 bf16 A tile per
 // stage (128 K, two 128-byte swizzle atoms).  One persistent CTA per SM, warp
